@@ -1,0 +1,153 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) fused Mixture-of-Experts layer.
+ *
+ * What it computes.  Fused MoE "combines token routing, data transfers and
+ * expert computation into a single batched operation on the GPU" ("AWS
+ * describes a fused MoE optimization for the NVIDIA Hopper architecture",
+ * body) and fuses "scaling, matrix multiplication and expert aggregation"
+ * ("AWS details MoE kernel fixes for SageMaker, upstreams them to vLLM",
+ * paragraph on the Triton backend).  For each token t:
+ *   logits[e] = hidden[t] . router_w[e] (+ router_bias[e])
+ *   p         = fp32 softmax over the E logits
+ *   ids       = the top_k experts by logit, descending, exact ties -> lower id
+ *   w[j]      = p[ids[j]] / sum_j' p[ids[j']]
+ *   for each slot j, expert e = ids[j]:
+ *       g = W1[e] x, u = W3[e] x   (W1 = rows [0,I) of w13[e], W3 = rows [I,2I))
+ *       h = SiLU(g) * u            (rounded to bf16, or E4M3 on the FP8 path)
+ *       y = W2[e] h
+ *   out[t] = bf16( sum_j w[j] * y_j )   (fp32 sum in slot order j = 0..top_k-1)
+ * The Hopper "Swap-AB" operand swap the pages describe ("AWS Unveils MoE
+ * Kernel Optimizations...", Swap-AB section) becomes a per-expert choice of
+ * tcgen05 orientation inside the library: experts with few tokens put the
+ * weight rows in the MMA's M slot and the tokens in N; experts with many
+ * tokens use the normal orientation.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_host are host memory (pinned for asynchrony); every
+ *    other pointer is device memory owned by the caller.  The library never
+ *    allocates or frees memory on these calls; scratch space comes from the
+ *    caller's workspace (moe_workspace_size).
+ *  - All device pointers must be 16-byte aligned.  Matrices are row-major and
+ *    densely packed.  bf16 = IEEE bfloat16 bit patterns (uint16); E4M3 = OCP
+ *    FP8 E4M3FN codes (uint8).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream: they enqueue kernels
+ *    and return.  Argument errors are returned synchronously and nothing is
+ *    enqueued.  Errors found on the device (a wait that timed out, an expert
+ *    id out of range) are recorded in the workspace's status word and read
+ *    with moe_get_status.
+ *  - Shapes are runtime values; nothing is specialised per T (the pages'
+ *    lesson about per-token-count JIT recompiles, "AWS details MoE kernel
+ *    fixes...", third fix).  Results are deterministic: identical inputs give
+ *    bit-identical outputs.
+ *  - Limits: 1 <= T, T*top_k <= 2^24; 1 <= E <= 1024; 1 <= top_k <= min(E, 32);
+ *    H and I multiples of 128 with 128 <= H <= 8192, 128 <= I <= 16384.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_DTYPE_BF16 = 0,     /* bf16 weights and activations, fp32 accumulate, bf16 out */
+  MOE_DTYPE_FP8_E4M3 = 1  /* E4M3 weights (one fp32 scale per expert matrix), dynamic
+                             per-tensor E4M3 activations and intermediate, bf16 out */
+} moe_dtype_t;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* NULL pointer, bad dtype, top_k out of range */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* a size outside the limits above */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 3,
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device-side wait expired */
+  MOE_ERR_DEVICE_BOUNDS = 6,      /* an expert id outside [0, E) reached moe_align */
+  MOE_ERR_MISALIGNED = 7          /* a pointer is not 16-byte aligned */
+} moe_status_t;
+
+/* Optional outputs of moe_forward for checking and profiling; every field may
+ * be NULL.  Device pointers unless noted. */
+typedef struct {
+  int32_t *topk_ids;   /* [T, top_k] expert ids, slot order */
+  float *topk_w;       /* [T, top_k] renormalised fp32 weights */
+  int32_t *counts;     /* [E] assignments per expert */
+  int32_t *offsets;    /* [E+1] exclusive prefix sum of counts */
+  int32_t *perm;       /* [T*top_k] flat index t*top_k+j, grouped by expert, ascending inside */
+  int32_t *inv_perm;   /* [T*top_k] inverse of perm */
+  void *inter;         /* [T*top_k, I] intermediate h in perm order (bf16 or E4M3 codes) */
+  float *act_scales;   /* [2] FP8 path: s1 (activations), s2 (intermediate) */
+  void **stage_events; /* host array of 8 cudaEvent_t recorded on `stream` at the stage
+                          boundaries: start, router, align, gather, w13, requant, w2, combine */
+  int force_orient;    /* 0 = per-expert choice, 1 = swap-AB for all experts,
+                          2 = normal orientation for all experts (testing) */
+} moe_debug_out_t;
+
+/* Bytes of workspace moe_forward needs for this shape (0 if the shape is
+ * outside the limits).  The workspace holds routing results, the grouped
+ * activations, the intermediate and the per-slot fp32 down-projection rows. */
+size_t moe_workspace_size(int T, int H, int E, int I, int top_k, int dtype);
+
+/* Zero the workspace's status header (256 bytes).  Call once on a fresh
+ * workspace before its first use. */
+moe_status_t moe_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* The whole layer.
+ *   hidden     [T, H] bf16                 router_w   [E, H] bf16
+ *   router_bias[E] fp32 or NULL: added to the logits before the softmax
+ *   w13        [E, 2I, H] bf16 or E4M3     w2         [E, H, I] bf16 or E4M3
+ *   w13_scale, w2_scale [E] fp32 (FP8 only, else NULL): weight = code * scale
+ *   out        [T, H] bf16, written fully
+ *   workspace  >= moe_workspace_size(...) bytes, initialised by moe_workspace_init
+ *   dbg        NULL in production
+ * Errors: MOE_ERR_INVALID_ARG / UNSUPPORTED_SHAPE / MISALIGNED /
+ * WORKSPACE_TOO_SMALL before any launch; MOE_ERR_CUDA if a launch fails. */
+moe_status_t moe_forward(const void *hidden, const void *router_w, const float *router_bias,
+                         const void *w13, const void *w2, const float *w13_scale,
+                         const float *w2_scale, int T, int H, int E, int I, int top_k, int dtype,
+                         void *out, void *workspace, size_t workspace_bytes,
+                         moe_debug_out_t *dbg, void *stream);
+
+/* moe_forward with host-side activations: copies hidden_host [T, H] bf16
+ * (pinned host memory) into the workspace, runs the layer, and copies the
+ * result into out_host [T, H] bf16 (pinned host memory), all enqueued on
+ * `stream`.  The caller synchronises the stream before reading out_host.
+ * Weights stay device pointers. */
+moe_status_t moe_forward_hostio(const void *hidden_host, const void *router_w,
+                                const float *router_bias, const void *w13, const void *w2,
+                                const float *w13_scale, const float *w2_scale, int T, int H,
+                                int E, int I, int top_k, int dtype, void *out_host,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Router only: topk_ids [T, top_k] int32 and topk_w [T, top_k] fp32 (device),
+ * same definition as in moe_forward.  Uses the workspace of moe_forward's
+ * shape (moe_workspace_size with the same T, H, E, top_k; any I >= 128). */
+moe_status_t moe_route(const void *hidden, const void *router_w, const float *router_bias,
+                       int T, int H, int E, int top_k, int32_t *topk_ids, float *topk_w,
+                       void *workspace, size_t workspace_bytes, void *stream);
+
+/* Align only: group the T*top_k assignments in topk_ids by expert.
+ * counts [E], offsets [E+1], perm and inv_perm [T*top_k] (device, int32),
+ * bit-exact stable counting sort.  Ids outside [0, E) set
+ * MOE_ERR_DEVICE_BOUNDS in the status word and are skipped. */
+moe_status_t moe_align(const int32_t *topk_ids, int T, int E, int top_k, int32_t *counts,
+                       int32_t *offsets, int32_t *perm, int32_t *inv_perm, void *workspace,
+                       size_t workspace_bytes, void *stream);
+
+/* Synchronises `stream`, returns the first device-side error recorded in the
+ * workspace since the last call (MOE_OK if none) and clears it.  *info_out
+ * (may be NULL) receives where it happened. */
+moe_status_t moe_get_status(void *workspace, void *stream, uint32_t *info_out);
+
+/* Static description of a status code. */
+const char *moe_status_string(moe_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

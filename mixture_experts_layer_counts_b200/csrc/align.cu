@@ -1,0 +1,167 @@
+// moe_align: group the T*k (token, slot) assignments by expert, bit-exact.
+//
+// Output contract (unpadded): counts[e]; offsets = exclusive prefix sum of
+// counts (E+1 entries); perm[p] = flat index f = t*k + j of the p-th
+// assignment in expert-major order, ascending f inside an expert (a stable
+// counting sort); inv_perm[perm[p]] = p.  The same pass builds the tile
+// schedule of the grouped GEMMs (token chunks per expert, per orientation)
+// and, on the FP8 path, the per-tensor activation scale s1 = amax|x| / 448.
+//
+// One CTA of 1024 threads.  Each warp owns a contiguous slice of the flat
+// indices; a per-warp histogram (warp-match of equal experts, leader adds the
+// group size) gives every warp its starting position per expert, so the
+// scatter is stable without atomics.
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+__device__ int block_exclusive_scan(int v, int* tmp32, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, d);
+    if (lane >= d) incl += o;
+  }
+  if (lane == 31) tmp32[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = tmp32[lane];
+    int wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += o;
+    }
+    tmp32[lane] = wi - w;   // exclusive warp offsets
+    if (lane == 31) *total = wi;
+  }
+  __syncthreads();
+  const int r = tmp32[warp] + incl - v;
+  __syncthreads();
+  return r;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
+  extern __shared__ int sh[];
+  int* hist = sh;                       // [32][E]
+  __shared__ int tmp32[32];
+  __shared__ int total;
+  __shared__ float famax[32];
+  const int E = a.E;
+  const int A = a.T * a.k;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+
+  const int per = (A + 31) / 32;
+  const int beg = min(A, warp * per), end = min(A, beg + per);
+  for (int base = beg; base < end; base += 32) {
+    const int f = base + lane;
+    int e = f < end ? a.topk_ids[f] : -1;
+    if (e >= E || e < -1) {
+      report_status(a.hdr, MOE_DEVICE_BOUNDS, 0x100u);
+      e = -1;
+    }
+    const unsigned act = __ballot_sync(0xffffffffu, true);
+    const unsigned grp = __match_any_sync(act, e);
+    if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // counts, offsets, per-warp starting positions
+  int c = 0;
+  if (threadIdx.x < E)
+    for (int w = 0; w < 32; ++w) c += hist[w * E + threadIdx.x];
+  const int excl = block_exclusive_scan(threadIdx.x < E ? c : 0, tmp32, &total);
+  if (threadIdx.x < E) {
+    a.counts[threadIdx.x] = c;
+    a.offsets[threadIdx.x] = excl;
+    int run = excl;
+    for (int w = 0; w < 32; ++w) {
+      const int h = hist[w * E + threadIdx.x];
+      hist[w * E + threadIdx.x] = run;
+      run += h;
+    }
+  }
+  if (threadIdx.x == 0) a.offsets[E] = total;
+  __syncthreads();
+
+  // stable scatter
+  for (int base = beg; base < end; base += 32) {
+    const int f = base + lane;
+    int e = f < end ? a.topk_ids[f] : -1;
+    if (e >= E || e < -1) e = -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, e);
+    const int rank = __popc(grp & ((1u << lane) - 1u));
+    if (e >= 0) {
+      const int pos = hist[warp * E + e] + rank;
+      a.perm[pos] = f;
+      a.inv_perm[f] = pos;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
+    __syncwarp();
+  }
+
+  // tile schedule: swap-AB chunks of <= kSwapMaxTokens tokens for experts
+  // with count <= swap_max_count, normal-orientation tiles of kNormalTokens
+  // tokens for the rest.
+  const bool ex = threadIdx.x < E && c > 0;
+  const bool sw = ex && c <= a.swap_max_count;
+  const int nsw = sw ? (c + kSwapMaxTokens - 1) / kSwapMaxTokens : 0;
+  const int nno = (ex && !sw) ? (c + kNormalTokens - 1) / kNormalTokens : 0;
+  const int osw = block_exclusive_scan(nsw, tmp32, &total);
+  const int tsw = total;
+  __syncthreads();
+  const int ono = block_exclusive_scan(nno, tmp32, &total);
+  const int tno = total;
+  for (int i = 0; i < nsw; ++i) {
+    const int n0 = i * kSwapMaxTokens;
+    a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(kSwapMaxTokens, c - n0), 0);
+  }
+  for (int i = 0; i < nno; ++i) {
+    const int n0 = i * kNormalTokens;
+    a.chunks_normal[ono + i] = make_int4(threadIdx.x, excl + n0, min(kNormalTokens, c - n0), 0);
+  }
+  if (threadIdx.x == 0) {
+    a.hdr[kHdrChunksSwap] = static_cast<uint32_t>(tsw);
+    a.hdr[kHdrChunksNormal] = static_cast<uint32_t>(tno);
+  }
+
+  // FP8 activation scale: s1 = amax / 448 (one IEEE fp32 division); amax == 0 -> 1
+  if (a.amax_tok != nullptr) {
+    float m = 0.f;
+    for (int t = threadIdx.x; t < a.T; t += blockDim.x) m = fmaxf(m, a.amax_tok[t]);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if (lane == 0) famax[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float mm = 0.f;
+      for (int w = 0; w < 32; ++w) mm = fmaxf(mm, famax[w]);
+      const float s1 = mm == 0.f ? 1.0f : __fdiv_rn(mm, 448.0f);
+      a.hdr[kHdrScaleS1] = __float_as_uint(s1);
+    }
+  }
+}
+
+cudaError_t launch_align(const AlignArgs& a, cudaStream_t st) {
+  const size_t smem = static_cast<size_t>(32) * a.E * sizeof(int);
+  cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       static_cast<int>(smem));
+  align_kernel<<<1, 1024, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,363 @@
+// C ABI of the fused MoE layer: argument checks, workspace carve-up,
+// per-expert orientation policy, tensor maps and the launch sequence.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "moe.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int device_sm_count() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+// Experts with at most this many tokens run swap-AB (weights in M, tokens in
+// N); heavier experts run the normal orientation.  MOE_SWAP_MAX_TOKENS
+// overrides it (for measurements), clamped to [0, kSwapMaxTokens].
+int swap_threshold() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = std::getenv("MOE_SWAP_MAX_TOKENS");
+    int t = s ? std::atoi(s) : kSwapMaxTokens;
+    v = t < 0 ? 0 : (t > kSwapMaxTokens ? kSwapMaxTokens : t);
+  }
+  return v;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+moe_status_t check_shape(int T, int H, int E, int I, int k, int dtype) {
+  if (dtype != MOE_DTYPE_BF16 && dtype != MOE_DTYPE_FP8_E4M3) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > kMaxExperts) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (k < 1 || k > E || k > kMaxTopK) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || static_cast<long long>(T) * k > (1LL << 24)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (H < 128 || H > 8192 || H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (I < 128 || I > 16384 || I % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+moe_status_t make_tmap(CUtensorMap* m, const void* base, bool fp8, int inner, long long rows,
+                       int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return MOE_ERR_CUDA;
+  const int esize = fp8 ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(inner) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kAtomBytes / esize), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                  \
+  do {                                 \
+    moe_status_t s_ = (expr);          \
+    if (s_ != MOE_OK) return s_;       \
+  } while (0)
+
+void record(moe_debug_out_t* dbg, int i, cudaStream_t st) {
+  if (dbg && dbg->stage_events && dbg->stage_events[i])
+    cudaEventRecord(static_cast<cudaEvent_t>(dbg->stage_events[i]), st);
+}
+
+moe_status_t forward_impl(const void* hidden, const void* router_w, const float* router_bias,
+                          const void* w13, const void* w2, const float* w13_scale,
+                          const float* w2_scale, int T, int H, int E, int I, int k, int dtype,
+                          void* out, void* ws, size_t ws_bytes, moe_debug_out_t* dbg,
+                          cudaStream_t st) {
+  MOE_TRY(check_shape(T, H, E, I, k, dtype));
+  const bool fp8 = dtype == MOE_DTYPE_FP8_E4M3;
+  if (!hidden || !router_w || !w13 || !w2 || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!w13_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(router_w) || !aligned16(w13) || !aligned16(w2) ||
+      !aligned16(out) || !aligned16(ws) || (router_bias && (reinterpret_cast<uintptr_t>(router_bias) & 3u)))
+    return MOE_ERR_MISALIGNED;
+  const Layout L = make_layout(T, H, E, I, k, fp8);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  const int A = T * k;
+  uint32_t* hdr = at<uint32_t>(ws, L.header);
+
+  int tau = swap_threshold();
+  if (dbg && dbg->force_orient == 1) tau = INT_MAX;
+  if (dbg && dbg->force_orient == 2) tau = 0;
+  if (H % 256 != 0) tau = INT_MAX;   // the normal-orientation w2 tile is 256 rows of H
+  const bool any_swap = tau > 0;
+  const bool any_normal = T > tau;
+
+  // tensor maps (weights and grouped activations), built before any launch
+  CUtensorMap tw13s, tw13n, tw2s, tw2n, txs, txn, tis, tin;
+  const long long w13_rows = static_cast<long long>(E) * 2 * I;
+  const long long w2_rows = static_cast<long long>(E) * H;
+  void* xperm = at<void>(ws, L.xperm);
+  void* inter = at<void>(ws, L.inter);
+  if (any_swap) {
+    MOE_TRY(make_tmap(&tw13s, w13, fp8, H, w13_rows, gemm_weight_box_rows(Orient::kSwap, Proj::kW13)));
+    MOE_TRY(make_tmap(&tw2s, w2, fp8, I, w2_rows, gemm_weight_box_rows(Orient::kSwap, Proj::kW2)));
+    MOE_TRY(make_tmap(&txs, xperm, fp8, H, A, gemm_token_box_rows(Orient::kSwap)));
+    MOE_TRY(make_tmap(&tis, inter, fp8, I, A, gemm_token_box_rows(Orient::kSwap)));
+  }
+  if (any_normal) {
+    MOE_TRY(make_tmap(&tw13n, w13, fp8, H, w13_rows, gemm_weight_box_rows(Orient::kNormal, Proj::kW13)));
+    MOE_TRY(make_tmap(&tw2n, w2, fp8, I, w2_rows, gemm_weight_box_rows(Orient::kNormal, Proj::kW2)));
+    MOE_TRY(make_tmap(&txn, xperm, fp8, H, A, gemm_token_box_rows(Orient::kNormal)));
+    MOE_TRY(make_tmap(&tin, inter, fp8, I, A, gemm_token_box_rows(Orient::kNormal)));
+  }
+
+  record(dbg, 0, st);
+  RouterArgs ra{static_cast<const __nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(router_w),
+                router_bias, T, H, E, k,
+                at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
+                at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
+                at<unsigned char>(ws, L.cand), hdr};
+  MOE_TRY(cuda_status(launch_router(ra, st)));
+  record(dbg, 1, st);
+
+  AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
+               at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
+               at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
+               tau, fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr};
+  MOE_TRY(cuda_status(launch_align(aa, st)));
+  record(dbg, 2, st);
+
+  MOE_TRY(cuda_status(launch_gather(static_cast<const __nv_bfloat16*>(hidden), at<int32_t>(ws, L.perm),
+                                    A, k, H, fp8, hdr, xperm, st)));
+  record(dbg, 3, st);
+
+  const int grid = device_sm_count() < kMaxGrid ? device_sm_count() : kMaxGrid;
+  GemmArgs g13{};
+  g13.katoms = H * (fp8 ? 1 : 2) / kAtomBytes;
+  g13.w_rows_per_expert = 2 * I;
+  g13.up_offset = I;
+  g13.out = fp8 ? at<void>(ws, L.h32) : inter;
+  g13.ld_out = I;
+  g13.perm = at<int32_t>(ws, L.perm);
+  g13.topk_w = at<float>(ws, L.topk_w);
+  g13.num_assign = A;
+  g13.wscale = w13_scale;
+  g13.act_scale = hdr + kHdrScaleS1;
+  g13.hdr = hdr;
+  float* amax_cta = at<float>(ws, L.amax_cta);
+  if (any_swap) {
+    GemmArgs g = g13;
+    g.chunks = at<int4>(ws, L.chunks_swap);
+    g.nchunks = hdr + kHdrChunksSwap;
+    g.mtiles = I / kTileM;
+    g.amax_cta = amax_cta;
+    MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW13, fp8, tw13s, txs, g, grid, st)));
+  }
+  if (any_normal) {
+    GemmArgs g = g13;
+    g.chunks = at<int4>(ws, L.chunks_normal);
+    g.nchunks = hdr + kHdrChunksNormal;
+    g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
+    g.amax_cta = amax_cta + (any_swap ? grid : 0);
+    MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
+  }
+  record(dbg, 4, st);
+  if (fp8) {
+    const int n_cta = (any_swap ? grid : 0) + (any_normal ? grid : 0);
+    MOE_TRY(cuda_status(launch_requant(at<float>(ws, L.h32), amax_cta, n_cta,
+                                       static_cast<size_t>(A) * I, hdr, static_cast<uint8_t*>(inter), st)));
+  }
+  record(dbg, 5, st);
+
+  GemmArgs g2 = g13;
+  g2.katoms = I * (fp8 ? 1 : 2) / kAtomBytes;
+  g2.w_rows_per_expert = H;
+  g2.up_offset = 0;
+  g2.out = at<void>(ws, L.ysc);
+  g2.ld_out = H;
+  g2.wscale = w2_scale;
+  g2.act_scale = hdr + kHdrScaleS2;
+  g2.amax_cta = nullptr;
+  if (any_swap) {
+    GemmArgs g = g2;
+    g.chunks = at<int4>(ws, L.chunks_swap);
+    g.nchunks = hdr + kHdrChunksSwap;
+    g.mtiles = H / kTileM;
+    MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, fp8, tw2s, tis, g, grid, st)));
+  }
+  if (any_normal) {
+    GemmArgs g = g2;
+    g.chunks = at<int4>(ws, L.chunks_normal);
+    g.nchunks = hdr + kHdrChunksNormal;
+    g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
+    MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
+  }
+  record(dbg, 6, st);
+  MOE_TRY(cuda_status(launch_combine(at<float>(ws, L.ysc), T, k, H, static_cast<__nv_bfloat16*>(out), st)));
+  record(dbg, 7, st);
+
+  if (dbg) {
+    auto cp = [&](void* dst, size_t off, size_t bytes) -> cudaError_t {
+      return dst ? cudaMemcpyAsync(dst, static_cast<char*>(ws) + off, bytes, cudaMemcpyDeviceToDevice, st)
+                 : cudaSuccess;
+    };
+    MOE_TRY(cuda_status(cp(dbg->topk_ids, L.topk_ids, static_cast<size_t>(A) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->topk_w, L.topk_w, static_cast<size_t>(A) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->counts, L.counts, static_cast<size_t>(E) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->offsets, L.offsets, static_cast<size_t>(E + 1) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->perm, L.perm, static_cast<size_t>(A) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->inv_perm, L.inv_perm, static_cast<size_t>(A) * 4)));
+    MOE_TRY(cuda_status(cp(dbg->inter, L.inter, static_cast<size_t>(A) * I * (fp8 ? 1 : 2))));
+    if (dbg->act_scales)
+      MOE_TRY(cuda_status(cudaMemcpyAsync(dbg->act_scales, hdr + kHdrScaleS1, 8, cudaMemcpyDeviceToDevice, st)));
+  }
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_size(int T, int H, int E, int I, int top_k, int dtype) {
+  if (check_shape(T, H, E, I, top_k, dtype) != MOE_OK) return 0;
+  return make_layout(T, H, E, I, top_k, dtype == MOE_DTYPE_FP8_E4M3).total;
+}
+
+moe_status_t moe_workspace_init(void* workspace, size_t workspace_bytes, void* stream) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  if (workspace_bytes < static_cast<size_t>(kHeaderBytes)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  return cuda_status(cudaMemsetAsync(workspace, 0, kHeaderBytes, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const void* hidden, const void* router_w, const float* router_bias,
+                         const void* w13, const void* w2, const float* w13_scale,
+                         const float* w2_scale, int T, int H, int E, int I, int top_k, int dtype,
+                         void* out, void* workspace, size_t workspace_bytes, moe_debug_out_t* dbg,
+                         void* stream) {
+  return forward_impl(hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I,
+                      top_k, dtype, out, workspace, workspace_bytes, dbg,
+                      static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
+                                const float* router_bias, const void* w13, const void* w2,
+                                const float* w13_scale, const float* w2_scale, int T, int H, int E,
+                                int I, int top_k, int dtype, void* out_host, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  MOE_TRY(check_shape(T, H, E, I, top_k, dtype));
+  if (!hidden_host || !out_host || !workspace) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(T, H, E, I, top_k, dtype == MOE_DTYPE_FP8_E4M3);
+  if (workspace_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* din = at<void>(workspace, L.staging_in);
+  void* dout = at<void>(workspace, L.staging_out);
+  const size_t bytes = static_cast<size_t>(T) * H * 2;
+  MOE_TRY(cuda_status(cudaMemcpyAsync(din, hidden_host, bytes, cudaMemcpyHostToDevice, st)));
+  MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
+                       dtype, dout, workspace, workspace_bytes, nullptr, st));
+  return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
+}
+
+moe_status_t moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,
+                       int H, int E, int top_k, int32_t* topk_ids, float* topk_w, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  MOE_TRY(check_shape(T, H, E, 128, top_k, MOE_DTYPE_BF16));
+  if (!hidden || !router_w || !topk_ids || !topk_w || !workspace) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(router_w) || !aligned16(workspace)) return MOE_ERR_MISALIGNED;
+  const Layout L = make_layout(T, H, E, 128, top_k, false);
+  if (workspace_bytes < L.cand + static_cast<size_t>(T) * E * 16) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  RouterArgs ra{static_cast<const __nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(router_w),
+                router_bias, T, H, E, top_k,
+                at<float>(workspace, L.logits), at<float>(workspace, L.xnorm),
+                at<float>(workspace, L.wnorm), at<float>(workspace, L.amax_tok), topk_ids, topk_w,
+                at<unsigned char>(workspace, L.cand), at<uint32_t>(workspace, L.header)};
+  return cuda_status(launch_router(ra, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t* counts,
+                       int32_t* offsets, int32_t* perm, int32_t* inv_perm, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (E < 1 || E > kMaxExperts || top_k < 1 || top_k > kMaxTopK || T < 1 ||
+      static_cast<long long>(T) * top_k > (1LL << 24))
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!topk_ids || !counts || !offsets || !perm || !inv_perm || !workspace) return MOE_ERR_INVALID_ARG;
+  const Layout L = make_layout(T, 128, E, 128, top_k, false);
+  if (workspace_bytes < L.chunks_normal + static_cast<size_t>(L.max_chunks_normal) * 16)
+    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  AlignArgs aa{topk_ids, T, E, top_k, counts, offsets, perm, inv_perm,
+               at<int4>(workspace, L.chunks_swap), at<int4>(workspace, L.chunks_normal),
+               swap_threshold(), nullptr, at<uint32_t>(workspace, L.header)};
+  return cuda_status(launch_align(aa, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_status(void* workspace, void* stream, uint32_t* info_out) {
+  if (!workspace) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (h[0] != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(h), st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (info_out) *info_out = h[1];
+  return static_cast<moe_status_t>(h[0]);
+}
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE_BOUNDS: return "expert id out of range";
+    case MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

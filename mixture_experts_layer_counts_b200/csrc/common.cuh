@@ -1,0 +1,103 @@
+// Shared definitions of the fused-MoE CUDA library: status codes, tile
+// constants, the workspace layout and the device-side status word.
+#pragma once
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace moe {
+
+// Device status codes (same values as moe_status_t in include/moe.h).
+constexpr uint32_t MOE_DEVICE_OK = 0;
+constexpr uint32_t MOE_DEVICE_TIMEOUT = 5;
+constexpr uint32_t MOE_DEVICE_BOUNDS = 6;
+
+// Where a device wait gave up (low byte of the status info word).
+enum WaitSite : uint32_t {
+  kSiteProducerEmpty = 1,
+  kSiteMmaFull = 2,
+  kSiteMmaAccEmpty = 3,
+  kSiteEpiAccFull = 4,
+  kSiteDrainTma = 5,
+  kSiteDrainMma = 6,
+  kSiteGridBarrier = 7,
+};
+
+constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
+
+// Tile geometry.  One K atom is 128 bytes of a row: 64 bf16 or 128 E4M3.
+constexpr int kAtomBytes = 128;
+constexpr int kTileM = 128;            // rows of the A operand per MMA (M)
+constexpr int kSwapMaxTokens = 64;     // largest token chunk in swap-AB (N <= 64)
+constexpr int kTokenBox = 16;          // rows per TMA box of the token operand (swap-AB)
+constexpr int kNormalTokens = 128;     // token rows per tile in normal orientation (M)
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxGrid = 1024;          // persistent grids never exceed this
+
+// Header words at the start of the workspace (uint32 units).
+constexpr int kHdrStatus = 0;          // first device error code (sticky)
+constexpr int kHdrInfo = 1;            // where it happened
+constexpr int kHdrChunksSwap = 4;      // number of swap-AB token chunks
+constexpr int kHdrChunksNormal = 5;    // number of normal-orientation token tiles
+constexpr int kHdrUncertain = 6;       // tokens whose router ordering needed fp64 / exact
+constexpr int kHdrScaleS1 = 8;         // fp32 bits: activation scale (FP8)
+constexpr int kHdrScaleS2 = 9;         // fp32 bits: intermediate scale (FP8)
+constexpr int kHdrBarrier = 12;        // grid barrier counter
+constexpr int kHeaderBytes = 256;
+
+__device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, uint32_t where) {
+  if (atomicCAS(status + kHdrStatus, 0u, code) == 0u) {
+    atomicExch(status + kHdrInfo, where);
+  }
+}
+
+// Byte offsets of every region of the caller-provided workspace.
+struct Layout {
+  size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand;
+  size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal;
+  size_t xperm, inter, h32, ysc, staging_in, staging_out, total;
+  int max_chunks_swap, max_chunks_normal;
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
+  Layout L{};
+  size_t A = static_cast<size_t>(T) * k;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 1024);
+    return o;
+  };
+  L.header = take(kHeaderBytes);
+  L.topk_ids = take(A * 4);
+  L.topk_w = take(A * 4);
+  L.logits = take(static_cast<size_t>(T) * E * 4);
+  L.xnorm = take(static_cast<size_t>(T) * 4);
+  L.wnorm = take(static_cast<size_t>(E) * 4);
+  L.amax_tok = take(static_cast<size_t>(T) * 4);
+  L.amax_cta = take(static_cast<size_t>(kMaxGrid) * 4);
+  L.cand = take(static_cast<size_t>(T) * E * 16);    // router fallback scratch
+  L.counts = take(static_cast<size_t>(E) * 4);
+  L.offsets = take(static_cast<size_t>(E + 1) * 4);
+  L.perm = take(A * 4);
+  L.inv_perm = take(A * 4);
+  L.max_chunks_swap = static_cast<int>(E + A / kSwapMaxTokens + 1);
+  L.max_chunks_normal = static_cast<int>(E + A / kNormalTokens + 1);
+  L.chunks_swap = take(static_cast<size_t>(L.max_chunks_swap) * 16);
+  L.chunks_normal = take(static_cast<size_t>(L.max_chunks_normal) * 16);
+  const size_t eb = fp8 ? 1 : 2;
+  L.xperm = take(A * H * eb);
+  L.inter = take(A * I * eb);
+  L.h32 = fp8 ? take(A * I * 4) : off;
+  L.ysc = take(A * H * 4);
+  L.staging_in = take(static_cast<size_t>(T) * H * 2);
+  L.staging_out = take(static_cast<size_t>(T) * H * 2);
+  L.total = off;
+  return L;
+}
+
+}  // namespace moe

@@ -1,0 +1,152 @@
+// Bandwidth-bound helper kernels of the layer:
+//   gather   x_perm[p] = hidden[perm[p] / k]  (bf16), or its per-tensor E4M3
+//            quantisation x / s1 (FP8 path; one IEEE fp32 division, RNE,
+//            saturating to +-448)
+//   requant  FP8 intermediate: s2 = max(per-CTA amax|h|) / 448, h_q = E4M3(h / s2)
+//   combine  out[t] = bf16(sum_{j<k} ysc[t*k + j]) in slot order, fp32 sum
+// All grids are sized from the SM count; 16-byte vector accesses.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+}  // namespace
+
+__global__ void gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm,
+                              int A, int k, int vpr, uint4* __restrict__ xperm) {
+  const int T = A / k;
+  const size_t n = static_cast<size_t>(A) * vpr;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / vpr);
+    const int c = static_cast<int>(i - static_cast<size_t>(p) * vpr);
+    const int t = min(max(perm[p] / k, 0), T - 1);   // perm is a bijection; clamp is a guard
+    xperm[i] = hidden[static_cast<size_t>(t) * vpr + c];
+  }
+}
+
+__global__ void gather_quant_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm,
+                                    int A, int k, int vpr, const uint32_t* __restrict__ hdr,
+                                    uint2* __restrict__ xq) {
+  const int T = A / k;
+  const float s1 = __uint_as_float(hdr[kHdrScaleS1]);
+  const size_t n = static_cast<size_t>(A) * vpr;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / vpr);
+    const int c = static_cast<int>(i - static_cast<size_t>(p) * vpr);
+    const int t = min(max(perm[p] / k, 0), T - 1);   // perm is a bijection; clamp is a guard
+    const uint4 v = hidden[static_cast<size_t>(t) * vpr + c];
+    const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(&v);
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 q = __bfloat1622float2(b[j]);
+      f[2 * j] = __fdiv_rn(q.x, s1);
+      f[2 * j + 1] = __fdiv_rn(q.y, s1);
+    }
+    xq[i] = make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
+  }
+}
+
+__global__ void requant_kernel(const float4* __restrict__ h32, const float* __restrict__ amax_cta,
+                               int n_cta, size_t n4, uint32_t* __restrict__ hdr,
+                               uint32_t* __restrict__ out) {
+  __shared__ float s_scale;
+  if (threadIdx.x < 32) {
+    float m = 0.f;
+    for (int i = threadIdx.x; i < n_cta; i += 32) m = fmaxf(m, amax_cta[i]);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
+    if (threadIdx.x == 0) {
+      const float s2 = m == 0.f ? 1.0f : __fdiv_rn(m, 448.0f);
+      s_scale = s2;
+      if (blockIdx.x == 0) hdr[kHdrScaleS2] = __float_as_uint(s2);
+    }
+  }
+  __syncthreads();
+  const float s2 = s_scale;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const float4 v = h32[i];
+    out[i] = pack_e4m3x4(__fdiv_rn(v.x, s2), __fdiv_rn(v.y, s2), __fdiv_rn(v.z, s2),
+                         __fdiv_rn(v.w, s2));
+  }
+}
+
+__global__ void combine_kernel(const float4* __restrict__ ysc, int T, int k, int h4,
+                               uint2* __restrict__ out) {
+  const size_t n = static_cast<size_t>(T) * h4;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / h4);
+    const int c = static_cast<int>(i - static_cast<size_t>(t) * h4);
+    const float4* src = ysc + static_cast<size_t>(t) * k * h4 + c;
+    float4 acc = src[0];
+    for (int j = 1; j < k; ++j) {
+      const float4 y = src[static_cast<size_t>(j) * h4];
+      acc.x += y.x;
+      acc.y += y.y;
+      acc.z += y.z;
+      acc.w += y.w;
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+  }
+}
+
+cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int A, int k, int H,
+                          bool fp8, const uint32_t* hdr, void* xperm, cudaStream_t st) {
+  const int vpr = H / 8;
+  const size_t n = static_cast<size_t>(A) * vpr;
+  const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
+  if (fp8)
+    gather_quant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(hidden), perm, A, k,
+                                              vpr, hdr, reinterpret_cast<uint2*>(xperm));
+  else
+    gather_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(hidden), perm, A, k, vpr,
+                                        reinterpret_cast<uint4*>(xperm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
+                           uint32_t* hdr, uint8_t* inter, cudaStream_t st) {
+  const size_t n4 = count / 4;
+  const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, static_cast<size_t>(sm_count()) * 8));
+  requant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(h32), amax_cta, n_cta, n4,
+                                       hdr, reinterpret_cast<uint32_t*>(inter));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
+                           cudaStream_t st) {
+  const int h4 = H / 4;
+  const size_t n = static_cast<size_t>(T) * h4;
+  const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
+  combine_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(ysc), T, k, h4,
+                                       reinterpret_cast<uint2*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,401 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM),
+// operands streamed into shared memory by TMA, persistent CTAs (one per SM).
+//
+// Orientation.  The Hopper "Swap-AB" fix described for vLLM's fused MoE
+// ("AWS details MoE kernel fixes for SageMaker...", body; "AWS Unveils MoE
+// Kernel Optimizations...", Swap-AB section) computes B^T A^T so the large
+// expert-weight dimension fills the instruction's fixed 64-row slot when a
+// decode batch has only a handful of tokens.  The sm_100a analogue:
+//   kSwap   : A (M = 128) = expert weight rows, B (N = 16..64) = the expert's
+//             tokens, D[weight row, token] in TMEM.  Used for experts with few
+//             tokens: every weight byte is streamed once, the MMA N is the
+//             token count rounded up to 16.
+//   kNormal : A (M = 128) = 128 tokens of one expert, B (N = 128 or 256) =
+//             weight rows, D[token, weight row].  Used for experts with many
+//             tokens (prefill-sized batches), where the MMA tile is full.
+// Projections.
+//   kW13 : two accumulators per tile, gate rows [i, i+.) and up rows
+//          [I+i, I+i+.) of w13[e], so one thread holds g and u of the same
+//          (token, i) and the epilogue forms h = SiLU(g) * u directly:
+//          bf16 path -> inter (bf16, RNE); FP8 path -> h (fp32) + per-CTA
+//          amax|h| for the per-tensor requantisation that follows.
+//   kW2  : one accumulator; the epilogue multiplies by the router weight
+//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), which
+//          the combine pass sums in slot order: deterministic, no atomics.
+//
+// Pipeline per CTA (192 threads):
+//   warp 0 lane 0  TMA producer: STAGES-deep ring of {A, B} tiles, 128-byte
+//                  K atoms in the 128B-swizzle layout, mbarrier complete_tx.
+//   warp 1 lane 0  MMA issuer: 4 MMAs (K = 16 bf16 / 32 E4M3 each) per atom
+//                  and accumulator; tcgen05.commit frees the smem slot; a
+//                  final commit hands the TMEM buffer to the epilogue.
+//   warps 2..5     epilogue: tcgen05.ld 32 lanes x 16 columns per warp
+//                  (warp w reads TMEM lanes 32*(w%4)..+31), math, stores.
+// Two TMEM accumulator buffers, so the epilogue of one tile overlaps the
+// mainloop of the next.  Every wait is bounded (see mbar_wait).
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace moe {
+
+template <Orient O, Proj P, bool FP8>
+struct Cfg {
+  static constexpr bool kSwap = O == Orient::kSwap;
+  static constexpr bool kDual = P == Proj::kW13;
+  static constexpr int kBN = kSwap ? kSwapMaxTokens : (kDual ? 128 : 256);   // max N
+  static constexpr int kATile = kTileM * kAtomBytes;
+  static constexpr int kBTile = kBN * kAtomBytes;
+  static constexpr int kNumA = (kSwap && kDual) ? 2 : 1;
+  static constexpr int kNumB = (!kSwap && kDual) ? 2 : 1;
+  static constexpr int kStageBytes = kNumA * kATile + kNumB * kBTile;
+  static constexpr int kStages = (kSwap && kDual) ? 5 : (kSwap ? 8 : 4);
+  static constexpr int kAccCols = (kDual ? 2 : 1) * kBN;       // per TMEM buffer
+  static constexpr int kTmemCols = 2 * kAccCols;               // 128, 256 or 512
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kAtomElems = FP8 ? 128 : 64;
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+  static_assert(kSmemBytes <= 232448, "shared memory");
+};
+
+constexpr int kThreads = 192;
+
+template <Orient O, Proj P, bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
+  using C = Cfg<O, P, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte aligned base for the swizzled tiles
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* tiles = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* drain = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 4 floats: epilogue warp amax
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_w);
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nunits = static_cast<int>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------- TMA producer --
+    const uint64_t pol_w = l2_policy_evict_first();
+    const uint64_t pol_x = l2_policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t armed = 0, armed_parity = 0;   // per-stage bookkeeping for the abort drain
+    bool ok = true;
+    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+      const int4 ch = a.chunks[u / a.mtiles];
+      const int mt = u % a.mtiles;
+      const int e = ch.x, p0 = ch.y, nv = ch.z;
+      uint32_t bytes;
+      int wrow0;
+      int nbox = 0;
+      if constexpr (C::kSwap) {
+        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
+        nbox = nvpad / kTokenBox;
+        bytes = C::kNumA * C::kATile + nvpad * kAtomBytes;
+        wrow0 = e * a.w_rows_per_expert + mt * kTileM;
+      } else {
+        bytes = C::kStageBytes;
+        wrow0 = e * a.w_rows_per_expert + mt * C::kBN;
+      }
+      for (int kb = 0; kb < a.katoms; ++kb) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = tiles + stage * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[stage], bytes);
+        armed |= 1u << stage;
+        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        const int kc = kb * C::kAtomElems;
+        if constexpr (C::kSwap) {
+          tma_load_2d(st, &tm_w, &full[stage], kc, wrow0, pol_w);
+          if constexpr (C::kDual) tma_load_2d(st + C::kATile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+          uint8_t* sb = st + C::kNumA * C::kATile;
+          for (int q = 0; q < nbox; ++q)
+            tma_load_2d(sb + q * kTokenBox * kAtomBytes, &tm_x, &full[stage], kc, p0 + q * kTokenBox, pol_x);
+        } else {
+          tma_load_2d(st, &tm_x, &full[stage], kc, p0, pol_x);
+          tma_load_2d(st + C::kATile, &tm_w, &full[stage], kc, wrow0, pol_w);
+          if constexpr (C::kDual)
+            tma_load_2d(st + C::kATile + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+        }
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      // let copies already in flight land before the CTA's smem is released
+      int dummy = 0;
+      for (int s = 0; s < C::kStages; ++s)
+        if ((armed >> s) & 1u)
+          mbar_wait(&full[s], (armed_parity >> s) & 1u, reinterpret_cast<volatile int*>(&dummy),
+                    a.hdr, kSiteDrainTma);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer --
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true;
+    bool issued = false;
+    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t accph = (it >> 1) & 1;
+      if (!mbar_wait(&acc_empty[buf], accph ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int4 ch = a.chunks[u / a.mtiles];
+      int n;
+      if constexpr (C::kSwap) {
+        n = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
+      } else {
+        n = C::kBN;
+      }
+      const uint32_t idesc = idesc_f32acc(FP8 ? 0u : 1u, kTileM, static_cast<uint32_t>(n));
+      const uint32_t d0 = tmem_base + buf * C::kAccCols;
+      const uint32_t d1 = d0 + C::kBN;
+      for (int kb = 0; kb < a.katoms; ++kb) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, a.hdr, kSiteMmaFull)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
+#pragma unroll
+        for (int kk = 0; kk < kAtomBytes / 32; ++kk) {
+          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t off = kk * 32;
+          if constexpr (C::kSwap) {
+            const uint32_t sb = st + C::kNumA * C::kATile;
+            mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(sb + off), idesc, acc);
+            if constexpr (C::kDual)
+              mma_ss<FP8>(d1, sdesc_sw128(st + C::kATile + off), sdesc_sw128(sb + off), idesc, acc);
+          } else {
+            mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(st + C::kATile + off), idesc, acc);
+            if constexpr (C::kDual)
+              mma_ss<FP8>(d1, sdesc_sw128(st + off), sdesc_sw128(st + C::kATile + C::kBTile + off),
+                          idesc, acc);
+          }
+        }
+        issued = true;
+        mma_commit(&empty[stage]);
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (ok) mma_commit(&acc_full[buf]);
+    }
+    if (!ok && issued) {
+      int dummy = 0;
+      mma_commit(drain);
+      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), a.hdr, kSiteDrainMma);
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------------------ epilogue --
+    const int q = warp & 3;               // TMEM lane quadrant of this warp
+    const int row = q * 32 + lane;        // accumulator row held by this thread
+    float amax = 0.f;
+    int it = 0;
+    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t accph = (it >> 1) & 1;
+      if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull)) break;
+      tc_fence_after();
+      const int4 ch = a.chunks[u / a.mtiles];
+      const int mt = u % a.mtiles;
+      const int e = ch.x, p0 = ch.y, nv = ch.z;
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
+      float scale = 1.f;
+      if constexpr (FP8) scale = a.wscale[e] * __uint_as_float(*a.act_scale);
+
+      if constexpr (C::kSwap && C::kDual) {
+        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
+        const int irow = mt * kTileM + row;
+        for (int c0 = 0; c0 < nvpad; c0 += 16) {
+          float g[16], uu[16];
+          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, g, uu);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < nv) {
+              const float gg = g[j] * scale, uv = uu[j] * scale;
+              const float h = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
+              const size_t o = static_cast<size_t>(p0 + n) * a.ld_out + irow;
+              if constexpr (FP8) {
+                static_cast<float*>(a.out)[o] = h;
+                amax = fmaxf(amax, fabsf(h));
+              } else {
+                static_cast<__nv_bfloat16*>(a.out)[o] = __float2bfloat16_rn(h);
+              }
+            }
+          }
+        }
+      } else if constexpr (C::kSwap) {
+        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
+        const int hrow = mt * kTileM + row;
+        for (int c0 = 0; c0 < nvpad; c0 += 16) {
+          float y[16];
+          tmem_ld16_wait(tbase + c0, y);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            const int f = n < nv ? a.perm[p0 + n] : -1;
+            if (f >= 0 && f < a.num_assign) {
+              const float wt = a.topk_w[f];
+              static_cast<float*>(a.out)[static_cast<size_t>(f) * a.ld_out + hrow] = y[j] * scale * wt;
+            }
+          }
+        }
+      } else if constexpr (C::kDual) {
+        const bool valid = row < nv;
+        const int p = p0 + row;
+        const int i0 = mt * C::kBN;
+        for (int c0 = 0; c0 < C::kBN; c0 += 16) {
+          float g[16], uu[16];
+          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, g, uu);
+          if (valid) {
+            float h[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const float gg = g[j] * scale, uv = uu[j] * scale;
+              h[j] = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
+            }
+            const size_t o = static_cast<size_t>(p) * a.ld_out + i0 + c0;
+            if constexpr (FP8) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + o);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                dst[j] = make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h[4 * j]), fabsf(h[4 * j + 1])),
+                                         fmaxf(fabsf(h[4 * j + 2]), fabsf(h[4 * j + 3]))));
+              }
+            } else {
+              uint4 pk[2];
+              uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(h[2 * j], h[2 * j + 1]);
+                pw[j] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o);
+              dst[0] = pk[0];
+              dst[1] = pk[1];
+            }
+          }
+        }
+      } else {
+        int f = row < nv ? a.perm[p0 + row] : -1;
+        const bool valid = f >= 0 && f < a.num_assign;
+        float wt = 0.f;
+        if (valid) wt = a.topk_w[f] * scale;
+        const int h0 = mt * C::kBN;
+        for (int c0 = 0; c0 < C::kBN; c0 += 16) {
+          float y[16];
+          tmem_ld16_wait(tbase + c0, y);
+          if (valid) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                                    static_cast<size_t>(f) * a.ld_out + h0 + c0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              dst[j] = make_float4(y[4 * j] * wt, y[4 * j + 1] * wt, y[4 * j + 2] * wt, y[4 * j + 3] * wt);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+    if constexpr (FP8 && C::kDual) {
+#pragma unroll
+      for (int d = 16; d > 0; d >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, d));
+      if (lane == 0) red[warp - 2] = amax;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if constexpr (FP8 && Cfg<O, P, FP8>::kDual) {
+    if (threadIdx.x == 0)
+      a.amax_cta[blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  }
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+template <Orient O, Proj P, bool FP8>
+static cudaError_t launch_one(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                              int grid, cudaStream_t st) {
+  using C = Cfg<O, P, FP8>;
+  auto kern = grouped_gemm_kernel<O, P, FP8>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (err != cudaSuccess) return err;
+  kern<<<grid, kThreads, C::kSmemBytes, st>>>(tw, tx, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tw, const CUtensorMap& tx,
+                        const GemmArgs& a, int grid, cudaStream_t st) {
+  if (o == Orient::kSwap) {
+    if (p == Proj::kW13)
+      return fp8 ? launch_one<Orient::kSwap, Proj::kW13, true>(tw, tx, a, grid, st)
+                 : launch_one<Orient::kSwap, Proj::kW13, false>(tw, tx, a, grid, st);
+    return fp8 ? launch_one<Orient::kSwap, Proj::kW2, true>(tw, tx, a, grid, st)
+               : launch_one<Orient::kSwap, Proj::kW2, false>(tw, tx, a, grid, st);
+  }
+  if (p == Proj::kW13)
+    return fp8 ? launch_one<Orient::kNormal, Proj::kW13, true>(tw, tx, a, grid, st)
+               : launch_one<Orient::kNormal, Proj::kW13, false>(tw, tx, a, grid, st);
+  return fp8 ? launch_one<Orient::kNormal, Proj::kW2, true>(tw, tx, a, grid, st)
+             : launch_one<Orient::kNormal, Proj::kW2, false>(tw, tx, a, grid, st);
+}
+
+int gemm_token_box_rows(Orient o) { return o == Orient::kSwap ? kTokenBox : kNormalTokens; }
+
+int gemm_weight_box_rows(Orient o, Proj p) {
+  if (o == Orient::kSwap) return kTileM;
+  return p == Proj::kW13 ? 128 : 256;
+}
+
+}  // namespace moe

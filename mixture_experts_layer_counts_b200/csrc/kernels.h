@@ -1,0 +1,80 @@
+// Host-side launch wrappers of the library's kernels (internal interface
+// between the C ABI in api.cu and the kernel translation units).
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace moe {
+
+struct RouterArgs {
+  const __nv_bfloat16* hidden;
+  const __nv_bfloat16* router_w;
+  const float* bias;
+  int T, H, E, k;
+  float* logits;
+  float* xnorm;
+  float* wnorm;
+  float* amax_tok;
+  int32_t* topk_ids;
+  float* topk_w;
+  unsigned char* cand;
+  uint32_t* hdr;
+};
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+
+struct AlignArgs {
+  const int32_t* topk_ids;
+  int T, E, k;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv_perm;
+  int4* chunks_swap;
+  int4* chunks_normal;
+  int swap_max_count;     // experts with count <= this run swap-AB
+  const float* amax_tok;  // FP8: per-token amax|x| (NULL on bf16)
+  uint32_t* hdr;
+};
+cudaError_t launch_align(const AlignArgs& a, cudaStream_t st);
+
+// x_perm[p, :] = hidden[perm[p] / k, :]   (bf16 copy, or E4M3 of x / s1 on FP8)
+cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int A, int k, int H,
+                          bool fp8, const uint32_t* hdr, void* xperm, cudaStream_t st);
+
+// FP8: s2 = max(amax_cta[0..n)) / 448, inter = E4M3(h32 / s2)
+cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
+                           uint32_t* hdr, uint8_t* inter, cudaStream_t st);
+
+// out[t, :] = bf16( sum_{j<k} ysc[t*k + j, :] ), j ascending
+cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
+                           cudaStream_t st);
+
+struct GemmArgs {
+  const int4* chunks;
+  const uint32_t* nchunks;     // header word holding the chunk count
+  int mtiles;                  // weight tiles per chunk
+  int katoms;                  // K / 128 bytes
+  int w_rows_per_expert;       // rows of one expert in the 2-D weight view
+  int up_offset;               // w13: row offset of the up half (= I)
+  void* out;                   // w13: inter (bf16) or h32 (fp32, FP8); w2: ysc (fp32)
+  int ld_out;
+  const int32_t* perm;
+  const float* topk_w;
+  int num_assign;              // T * top_k (bounds of perm values)
+  const float* wscale;         // FP8 per-expert weight scale
+  const uint32_t* act_scale;   // FP8: header word with s1 (w13) or s2 (w2)
+  float* amax_cta;             // FP8 w13: per-CTA amax|h|
+  uint32_t* hdr;
+};
+
+enum class Orient { kSwap, kNormal };
+enum class Proj { kW13, kW2 };
+cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tm_w,
+                        const CUtensorMap& tm_x, const GemmArgs& a, int grid, cudaStream_t st);
+int gemm_token_box_rows(Orient o);   // rows per TMA box of the token operand
+int gemm_weight_box_rows(Orient o, Proj p);
+
+}  // namespace moe

@@ -1,0 +1,434 @@
+// Router: logits, fp32 softmax, top-k (ties -> lower expert index),
+// renormalisation.
+//
+// The selection is defined on the exact real-valued logits of the bf16 inputs
+// (the pages give no precision for routing; exactness makes "bit-exact
+// routing" independent of summation order).  Three tiers:
+//   1. fp32 logits with a rigorous error bound.  Products of two bf16 values
+//      are exact in fp32, so each logit carries only summation error,
+//      |err| <= gamma_n * sum|x*w| <= gamma_n * ||x|| * ||w|| (n = the
+//      longest chain of roundings: H/32 sequential FMAs per lane plus the
+//      5-level warp butterfly), plus one rounding for the bias.
+//   2. A token whose top-(k+1) ordering is not separated by twice that bound
+//      re-evaluates only its candidate experts in fp64 (bound ~1e-16 rel).
+//   3. Candidates still within 2x the fp64 bound of each other are ordered by
+//      their exact values, accumulated as 640-bit fixed-point integers.
+// Softmax and the renormalised weights are computed in fp32 from the fp32
+// logits, one warp per token with shuffle reductions.
+#include <cuda_bf16.h>
+
+#include <cfloat>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kLimbs = 20;      // 20 x 32-bit limbs: bit b <-> 2^(b - kExactOffset)
+constexpr int kExactOffset = 300;
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8]) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 t = __bfloat1622float2(p[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, m));
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
+}
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  return v;
+}
+
+// (value desc, index asc) total order used for top-k.
+__device__ __forceinline__ bool beats(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+// ---- exact fixed-point accumulation of bf16 products (tier 3) -------------
+// A bf16 value is sign * m * 2^q with m an 8-bit integer (hidden bit
+// included) and q = exponent_field - 134 (normal) or -133 (subnormal).
+__device__ __forceinline__ void bf16_parts(uint16_t b, uint32_t& m, int& q, uint32_t& s) {
+  s = b >> 15;
+  const uint32_t ef = (b >> 7) & 0xFFu;
+  const uint32_t f = b & 0x7Fu;
+  if (ef == 0) {
+    m = f;
+    q = -133;
+  } else {
+    m = f | 0x80u;
+    q = static_cast<int>(ef) - 134;
+  }
+}
+
+__device__ __forceinline__ void limb_add(long long (&acc)[kLimbs], uint64_t mag, int bitpos,
+                                         bool neg) {
+  const int li = bitpos >> 5;
+  const uint64_t v = mag << (bitpos & 31);   // mag < 2^24, shift < 32: fits 64 bits
+  const long long lo = static_cast<long long>(v & 0xFFFFFFFFull);
+  const long long hi = static_cast<long long>(v >> 32);
+  if (neg) {
+    acc[li] -= lo;
+    acc[li + 1] -= hi;
+  } else {
+    acc[li] += lo;
+    acc[li + 1] += hi;
+  }
+}
+
+// Exact logit of (token row x, expert row w) + bias, normalised limbs, in
+// every lane of the warp.
+__device__ void exact_logit(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w,
+                            float bias, int H, long long (&acc)[kLimbs]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int i = 0; i < kLimbs; ++i) acc[i] = 0;
+  for (int h = lane; h < H; h += 32) {
+    uint32_t mx, mw, sx, sw;
+    int qx, qw;
+    bf16_parts(x[h], mx, qx, sx);
+    bf16_parts(w[h], mw, qw, sw);
+    if (mx == 0 || mw == 0) continue;
+    limb_add(acc, static_cast<uint64_t>(mx) * mw, qx + qw + kExactOffset, (sx ^ sw) != 0);
+  }
+#pragma unroll
+  for (int i = 0; i < kLimbs; ++i) acc[i] = warp_sum_ll(acc[i]);
+  if (bias != 0.0f) {
+    const uint32_t b = __float_as_uint(bias);
+    const uint32_t ef = (b >> 23) & 0xFFu;
+    const uint32_t f = b & 0x7FFFFFu;
+    const uint32_t m = ef == 0 ? f : (f | 0x800000u);
+    const int q = ef == 0 ? -149 : static_cast<int>(ef) - 150;
+    limb_add(acc, m, q + kExactOffset, (b >> 31) != 0);
+  }
+  // carry-normalise: limbs 0..18 in [0, 2^32), the top limb keeps the sign
+#pragma unroll
+  for (int i = 0; i < kLimbs - 1; ++i) {
+    const long long c = acc[i] >> 32;   // arithmetic shift = floor division
+    acc[i] -= c * 4294967296LL;
+    acc[i + 1] += c;
+  }
+}
+
+__device__ __forceinline__ int exact_cmp(const long long (&a)[kLimbs], const long long (&b)[kLimbs]) {
+#pragma unroll
+  for (int i = kLimbs - 1; i >= 0; --i) {
+    if (a[i] != b[i]) return a[i] > b[i] ? 1 : -1;
+  }
+  return 0;
+}
+
+// fp64 logit (tier 2): exact products, fp64 sequential sums per lane, butterfly.
+__device__ double fp64_logit(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
+                             int H) {
+  const int lane = threadIdx.x & 31;
+  double acc = 0.0;
+  const uint4* xv = reinterpret_cast<const uint4*>(x);
+  const uint4* wv = reinterpret_cast<const uint4*>(w);
+  for (int c = lane; c < H / 8; c += 32) {
+    float xf[8], wf[8];
+    unpack8(xv[c], xf);
+    unpack8(wv[c], wf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc);
+  }
+  return warp_sum_d(acc);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Kernel 1: logits[t, e] = sum_h x[t,h] w[e,h] + b[e] in fp32, plus ||x_t||,
+// ||w_e|| for the error bound and per-token amax|x| for FP8 activation scale.
+// CTA = TT tokens x 8 experts (one expert per warp); hidden rows staged in smem.
+// ---------------------------------------------------------------------------
+template <int TT>
+__global__ void __launch_bounds__(256) router_logits_kernel(
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
+    const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
+  extern __shared__ uint4 sx[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * TT;
+  const int nt = min(TT, T - t0);
+  const int vpr = H / 8;   // 16-byte vectors per row
+  const uint4* hv = reinterpret_cast<const uint4*>(hidden);
+  for (int i = threadIdx.x; i < TT * vpr; i += blockDim.x) {
+    const int r = i / vpr;
+    sx[i] = r < nt ? hv[static_cast<size_t>(t0 + r) * vpr + (i - r * vpr)] : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
+
+  if (blockIdx.y == 0) {
+    for (int r = warp; r < nt; r += 8) {
+      float ss = 0.f, am = 0.f;
+      for (int c = lane; c < vpr; c += 32) {
+        float f[8];
+        unpack8(sx[r * vpr + c], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          ss = fmaf(f[i], f[i], ss);
+          am = fmaxf(am, fabsf(f[i]));
+        }
+      }
+      ss = warp_sum(ss);
+      am = warp_max(am);
+      if (lane == 0) {
+        xnorm[t0 + r] = sqrtf(ss);
+        amax_tok[t0 + r] = am;
+      }
+    }
+  }
+
+  const int e = blockIdx.y * 8 + warp;
+  if (e >= E) return;
+  float acc[TT];
+#pragma unroll
+  for (int i = 0; i < TT; ++i) acc[i] = 0.f;
+  float wsq = 0.f;
+  const uint4* wrow = reinterpret_cast<const uint4*>(router_w) + static_cast<size_t>(e) * vpr;
+  for (int c = lane; c < vpr; c += 32) {
+    float wf[8];
+    unpack8(wrow[c], wf);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) wsq = fmaf(wf[i], wf[i], wsq);
+#pragma unroll
+    for (int tt = 0; tt < TT; ++tt) {
+      float xf[8];
+      unpack8(sx[tt * vpr + c], xf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
+    }
+  }
+#pragma unroll
+  for (int tt = 0; tt < TT; ++tt) acc[tt] = warp_sum(acc[tt]);
+  wsq = warp_sum(wsq);
+  if (lane == 0) {
+    const float b = bias ? bias[e] : 0.f;
+    for (int tt = 0; tt < nt; ++tt) logits[static_cast<size_t>(t0 + tt) * E + e] = acc[tt] + b;
+    if (blockIdx.x == 0) wnorm[e] = sqrtf(wsq);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Kernel 2: one warp per token.  fp32 softmax, top-(k+1) by repeated warp
+// argmax, certification against the error bound, fallback tiers 2-3.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) router_topk_kernel(
+    const float* __restrict__ logits, const float* __restrict__ xnorm,
+    const float* __restrict__ wnorm, const float* __restrict__ bias,
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w, int T,
+    int H, int E, int k, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+    unsigned char* __restrict__ cand, uint32_t* __restrict__ hdr) {
+  constexpr int kPer = kMaxExperts / 32;
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int nper = (E + 31) / 32;
+  const float* row = logits + static_cast<size_t>(t) * E;
+  const float xn = xnorm[t];
+  const float gamma32 = static_cast<float>(H / 32 + 16) * 5.9604645e-08f * 1.0001f;
+
+  float v[kPer];
+  uint32_t taken = 0;
+  float rmax = 0.f, vmax = -FLT_MAX;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = -FLT_MAX;
+    if (i < nper && e < E) {
+      const float lv = row[e];
+      v[i] = isnan(lv) ? -FLT_MAX : lv;   // a NaN logit ranks last
+      const float b = bias ? fabsf(bias[e]) : 0.f;
+      const float r = (gamma32 * xn * wnorm[e] + 1.1920929e-07f * (fabsf(v[i]) + b)) * 1.001f;
+      rmax = fmaxf(rmax, r);
+      vmax = fmaxf(vmax, v[i]);
+    }
+  }
+  rmax = warp_max(rmax);
+  vmax = warp_max(vmax);
+  float se = 0.f;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i)
+    if (i < nper && lane + 32 * i < E) se += expf(v[i] - vmax);
+  se = warp_sum(se);
+
+  // top-(k+1) selection, warp-wide argmax per round
+  const int nsel = min(k + 1, E);
+  int sel_idx[kMaxTopK + 1];
+  float sel_v[kMaxTopK + 1];
+  for (int s = 0; s < nsel; ++s) {
+    float bv = -FLT_MAX;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = lane + 32 * i;
+      if (i < nper && e < E && !((taken >> i) & 1u) && beats(v[i], e, bv, bi)) {
+        bv = v[i];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, m);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, m);
+      if (beats(ov, oi, bv, bi)) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    sel_idx[s] = bi;
+    sel_v[s] = bv;
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+  }
+
+  bool certified = true;
+  if (rmax > 0.f) {
+    const double margin = 2.000001 * static_cast<double>(rmax);
+    for (int s = 0; s + 1 < nsel; ++s)
+      if (!(static_cast<double>(sel_v[s]) - static_cast<double>(sel_v[s + 1]) > margin))
+        certified = false;
+  }
+
+  int out[kMaxTopK];
+  if (certified) {
+    for (int j = 0; j < k; ++j) out[j] = sel_idx[j];
+  } else {
+    if (lane == 0) atomicAdd(hdr + kHdrUncertain, 1u);
+    // ---- tier 2: candidates re-evaluated in fp64 --------------------------
+    int* c_idx = reinterpret_cast<int*>(cand + static_cast<size_t>(t) * E * 16);
+    int* c_ord = c_idx + E;
+    double* c_val = reinterpret_cast<double*>(c_ord + E);
+    const double thr = static_cast<double>(sel_v[k - 1]) - 2.000001 * static_cast<double>(rmax);
+    int nc = 0;
+    for (int i = 0; i < nper; ++i) {
+      const int e = lane + 32 * i;
+      const bool is_c = e < E && static_cast<double>(v[i]) >= thr;
+      const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+      if (is_c) c_idx[nc + __popc(bal & ((1u << lane) - 1u))] = e;
+      nc += __popc(bal);
+    }
+    __syncwarp();
+    const double gamma64 = static_cast<double>(H / 32 + 16) * 1.1102230246251565e-16 * 1.0001;
+    double r64 = 0.0;
+    const __nv_bfloat16* xrow = hidden + static_cast<size_t>(t) * H;
+    for (int c = 0; c < nc; ++c) {
+      const int e = c_idx[c];
+      double d = fp64_logit(xrow, router_w + static_cast<size_t>(e) * H, H);
+      const double b = bias ? static_cast<double>(bias[e]) : 0.0;
+      d += b;
+      const double r = (gamma64 * xn * wnorm[e] + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
+      r64 = fmax(r64, r);
+      if (lane == 0) c_val[c] = d;
+    }
+    __syncwarp();
+    for (int c = lane; c < nc; c += 32) c_ord[c] = c;   // valid even if ranks collide (NaN)
+    __syncwarp();
+    for (int c = lane; c < nc; c += 32) {   // rank by (value desc, index asc)
+      const double vc = c_val[c];
+      const int ic = c_idx[c];
+      int rank = 0;
+      for (int j = 0; j < nc; ++j) {
+        const double vj = c_val[j];
+        rank += (vj > vc || (vj == vc && c_idx[j] < ic)) ? 1 : 0;
+      }
+      if (rank < nc) c_ord[rank] = c;
+    }
+    __syncwarp();
+    // ---- tier 3: clusters closer than the fp64 bound, ordered exactly -----
+    const double margin64 = 2.000001 * r64;
+    int got = 0, pos = 0;
+    const uint16_t* xbits = reinterpret_cast<const uint16_t*>(xrow);
+    while (got < k) {
+      int end = pos;
+      while (end + 1 < nc && !(c_val[c_ord[end]] - c_val[c_ord[end + 1]] > margin64)) ++end;
+      if (end == pos) {
+        out[got++] = c_idx[c_ord[pos]];
+        pos = end + 1;
+        continue;
+      }
+      const int need = min(end - pos + 1, k - got);
+      for (int q = 0; q < need; ++q) {
+        long long best[kLimbs];
+        int best_e = -1, best_slot = -1;
+        for (int m = pos; m <= end; ++m) {
+          const int e = c_idx[c_ord[m]];
+          if (e < 0) continue;   // already chosen
+          long long cur[kLimbs];
+          exact_logit(xbits, reinterpret_cast<const uint16_t*>(router_w) + static_cast<size_t>(e) * H,
+                      bias ? bias[e] : 0.f, H, cur);
+          int cmp = best_e < 0 ? 1 : exact_cmp(cur, best);
+          if (cmp > 0 || (cmp == 0 && e < best_e)) {
+#pragma unroll
+            for (int i = 0; i < kLimbs; ++i) best[i] = cur[i];
+            best_e = e;
+            best_slot = m;
+          }
+        }
+        out[got++] = best_e;
+        __syncwarp();
+        if (lane == 0) c_idx[c_ord[best_slot]] = -1;
+        __syncwarp();
+      }
+      pos = end + 1;
+    }
+  }
+
+  // renormalised weights of the selected experts (fp32 softmax values)
+  float p[kMaxTopK];
+  float psum = 0.f;
+  for (int j = 0; j < k; ++j) {
+    p[j] = expf(row[out[j]] - vmax) / se;
+    psum += p[j];
+  }
+  for (int j = lane; j < k; j += 32) {
+    topk_ids[static_cast<size_t>(t) * k + j] = out[j];
+    topk_w[static_cast<size_t>(t) * k + j] = p[j] / psum;
+  }
+}
+
+// ---------------------------------------------------------------------------
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
+  const int tt = a.T > 256 ? 16 : 8;
+  dim3 grid((a.T + tt - 1) / tt, (a.E + 7) / 8);
+  const size_t smem = static_cast<size_t>(tt) * a.H * 2;
+  if (tt == 16) {
+    cudaFuncSetAttribute(router_logits_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    router_logits_kernel<16><<<grid, 256, smem, st>>>(a.hidden, a.router_w, a.bias, a.T, a.H,
+                                                      a.E, a.logits, a.xnorm, a.wnorm, a.amax_tok);
+  } else {
+    cudaFuncSetAttribute(router_logits_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         static_cast<int>(smem));
+    router_logits_kernel<8><<<grid, 256, smem, st>>>(a.hidden, a.router_w, a.bias, a.T, a.H, a.E,
+                                                     a.logits, a.xnorm, a.wnorm, a.amax_tok);
+  }
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  router_topk_kernel<<<(a.T + 7) / 8, 256, 0, st>>>(a.logits, a.xnorm, a.wnorm, a.bias, a.hidden,
+                                                    a.router_w, a.T, a.H, a.E, a.k, a.topk_ids,
+                                                    a.topk_w, a.cand, a.hdr);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

