@@ -55,15 +55,91 @@ def assert_routing_equal(dbg, ref):
     assert np.abs(w - ref["weights"]).max() <= WEIGHT_ATOL
 
 
-def assert_output_close(out, ref, fp8, tokens=None):
+def bf16_rounding_ambiguity(inp, ref, tokens=None):
+    """bf16 results of the intermediate that fp32 arithmetic can legitimately give.
+
+    The GPU forms h = SiLU(g) * u in fp32 from fp32 tensor-core accumulators and
+    rounds it once to bf16; the oracle rounds its fp64 h once.  Where the exact
+    h lies closer to a bf16 rounding boundary than the kernel's fp32 arithmetic
+    resolves, more than one bf16 value is a correct result.  Error band of the
+    kernel's h:
+        band = 2^-19 |h| + 2^-21 (|SiLU'(g) u| S_g + |SiLU(g)| S_u)
+    with S_g = sum_k |x_k W1[i,k]|, S_u likewise: a few fp32 ulps of the
+    accumulated magnitudes (this term dominates under cancellation, g or u
+    much smaller than S) plus the SiLU's own fp32 error.  The valid results
+    are the bf16 roundings of [h - band, h + band].
+
+    Returns (amb: {perm position -> (lo, hi) arrays over I}, env [T, H]); env is
+    the largest change of the output the non-nearest valid results can cause:
+    env[t, o] = sum_j w[t,j] sum_i |W2[e][o, i]| * max(h_hi - r, r - h_lo).
+    """
+    from scipy.special import expit
+
+    from mixture_experts_layer_counts_b200.inputs import host_bits as hb
+    from oracle import bf16_bits_to_f64 as dec
+    from oracle import round_to_bf16
+
+    k = inp["top_k"]
+    x = dec(hb(inp["hidden"]))
+    T, H = x.shape
+    perm, off, w = ref["perm"], ref["offsets"], ref["weights"]
+    want = np.ones(T, bool) if tokens is None else np.isin(np.arange(T), tokens)
+    amb, env = {}, np.zeros((T, H))
+    for e in range(len(off) - 1):
+        rows = [p for p in range(off[e], off[e + 1]) if want[perm[p] // k]]
+        if not rows:
+            continue
+        W = dec(hb(inp["w13"][e]))
+        I = W.shape[0] // 2
+        Xe = x[perm[rows] // k]
+        g, u = Xe @ W[:I].T, Xe @ W[I:].T
+        Sg, Su = np.abs(Xe) @ np.abs(W[:I]).T, np.abs(Xe) @ np.abs(W[I:]).T
+        sig = expit(g)
+        s = g * sig
+        ds = sig * (1.0 + g * (1.0 - sig))
+        h = s * u
+        r = round_to_bf16(h)
+        band = 2.0 ** -19 * np.abs(h) + 2.0 ** -21 * (np.abs(ds * u) * Sg + np.abs(s) * Su)
+        lo, hi = round_to_bf16(h - band), round_to_bf16(h + band)
+        dev = np.maximum(hi - r, r - lo)
+        W2 = None
+        for ri, p in enumerate(rows):
+            amb[p] = (lo[ri], hi[ri])
+            a = dev[ri] > 0
+            if a.any():
+                W2 = dec(hb(inp["w2"][e])) if W2 is None else W2
+                f = perm[p]
+                env[f // k] += w[f // k, f % k] * (np.abs(W2[:, a]) @ dev[ri, a])
+    return amb, env
+
+
+def assert_inter_equal(dbg, ref, amb):
+    """GPU intermediate == oracle intermediate wherever the rounding is unique,
+    and one of the valid roundings (bf16_rounding_ambiguity) elsewhere."""
+    from mixture_experts_layer_counts_b200.inputs import host_bits as hb
+    from oracle import bf16_bits_to_f64 as dec
+
+    gi = dec(hb(dbg["inter"]))
+    ri = ref["inter"]
+    n_amb = n_diff = 0
+    for p, (lo, hi) in amb.items():
+        n_diff += int((gi[p] != ri[p]).sum())
+        n_amb += int((lo != hi).sum())
+        ok = (gi[p] >= lo) & (gi[p] <= hi)
+        assert ok.all(), f"intermediate row {p} outside its valid roundings at {np.nonzero(~ok)[0][:4]}"
+    return n_diff, n_amb
+
+
+def assert_output_close(out, ref, fp8, tokens=None, env=None):
     o = out.float().cpu().numpy().astype(np.float64)
     r = ref["out"]
     if tokens is not None:
         o, r = o[tokens], r[tokens]
+        env = None if env is None else env[tokens]
     if fp8:
         err = rel_l2(o, r)
         assert err <= 3e-2, f"FP8 relative L2 {err:.4g} > 3e-2"
         return err
-    v = bf16_tolerance_violation(o, r)
+    v = bf16_tolerance_violation(o, r, extra=env)
     assert v <= 1.0, f"bf16 tolerance exceeded: worst ratio {v:.3g}"
     return v
