@@ -1,0 +1,372 @@
+"""Benchmark of the fused MoE layer (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+
+A step is one call of the whole layer (router, align, gather, w13 GEMM with
+SiLU*up, [FP8 requant], w2 GEMM with router-weighted slot scatter, combine)
+on one batch of synthetic decode tokens whose inputs already sit in HBM.
+Each rank runs its own batch (independent decode batches, weights replicated,
+no data-path collective): weak scaling, value = all ranks' tokens / the
+slowest rank's device time.  Between timed steps L2 is flushed by writing a
+256 MiB buffer; each step is timed alone with CUDA events on the launch
+stream, and the flush is outside the events.
+
+Extra keys: us_per_layer, weight_bytes / weight_gbs (activated experts'
+weight bytes counted once per step), stages_us (per-kernel-stage device time
+from events the library records on the launch stream), roofline of the
+dominant kernel (w13 grouped GEMM, weight bytes of active experts / its
+measured time vs the measured HBM peak), e2e (same metric through the
+host-buffer C-ABI call with the H2D/D2H copies in the timed region),
+cpu_baseline (the fp64 oracle on a bounded token sample on the host cores),
+gpu_launches and clocks sampled with nvidia-smi during the timed region.
+
+--impl reference times the fp64 CPU oracle (the only other implementation of
+the layer; there is no installable reference package) on a bounded token
+sample per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from mixture_experts_layer_counts_b200.inputs import WORKLOADS, describe, make_inputs  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+REF_SAMPLE_TOKENS = 1          # tokens per --impl reference step
+CPU_BASELINE_TOKENS = 4        # tokens in the cpu_baseline sample
+FALLBACK_HBM_GBS = 6650.0
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_traffic(workload):
+    """ncu DRAM bytes per launch of the w13 kernel, if captured for this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(workload)
+    if not d:
+        return None
+    src = open(os.path.join(ROOT, "mixture_experts_layer_counts_b200", "csrc", "gemm.cu"), "rb").read()
+    if hashlib.sha256(src).hexdigest()[:16] != d.get("gemm_cu_sha"):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample_seconds(inp_host, wl, tokens):
+    """Wall time of one oracle call on a token sample (inputs already on host)."""
+    from oracle import moe_forward_ref
+
+    t0 = time.perf_counter()
+    moe_forward_ref(inp_host["hidden"], inp_host["router_w"], inp_host["bias"], inp_host["w13"],
+                    inp_host["w2"], wl["top_k"], wl["dtype"], inp_host["s13"], inp_host["s2"],
+                    tokens=tokens)
+    return time.perf_counter() - t0
+
+
+def host_copy(inp):
+    from mixture_experts_layer_counts_b200.inputs import host_bits
+
+    fp8 = inp["dtype"] == "fp8"
+    return dict(hidden=host_bits(inp["hidden"]), router_w=host_bits(inp["router_w"]),
+                bias=None if inp["router_bias"] is None else inp["router_bias"].float().cpu().numpy(),
+                w13=host_bits(inp["w13"]), w2=host_bits(inp["w2"]),
+                s13=inp["w13_scale"].cpu().numpy() if fp8 else None,
+                s2=inp["w2_scale"].cpu().numpy() if fp8 else None)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [p.get("num_threads") for p in threadpool_info() if p.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, wl, rank, world):
+    if rank != 0:
+        return
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(wl, dev, seed=wl["seed"])
+    host = host_copy(inp)
+    del inp
+    toks = list(range(REF_SAMPLE_TOKENS))
+    for _ in range(args.warmup):
+        oracle_sample_seconds(host, wl, toks)
+    times = [oracle_sample_seconds(host, wl, toks) for _ in range(args.steps)]
+    total = sum(times)
+    value = len(toks) * args.steps / total
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {describe(wl)}", "sample": f"{len(toks)} of {wl['T']} tokens"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"fp64 oracle, tokens 0..{len(toks) - 1} of the {args.workload} batch "
+                                   f"(full routing of all {wl['T']} tokens) per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+SWAP_MAX_TOKENS = 64   # the library's default swap-AB / normal threshold (tokens per expert)
+
+
+def launches_per_step(wl, T):
+    """Kernels one layer call launches: router (logits, top-k), align, gather,
+    w13 and w2 GEMMs (one per orientation in use), FP8 requant, combine."""
+    any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
+    n = 2 + 1 + 1 + 2 * (2 if any_normal else 1) + 1
+    return n + (1 if wl["dtype"] == "fp8" else 0)
+
+
+def run_ours(args, wl, rank, world, local):
+    from mixture_experts_layer_counts_b200 import layer
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    # each rank serves its own decode batch: rank-dependent hidden, shared weight seed
+    inp = make_inputs(wl, dev, seed=wl["seed"])
+    if world > 1:
+        from mixture_experts_layer_counts_b200.inputs import make_hidden
+
+        inp["hidden"] = make_hidden(wl, dev, seed=wl["seed"] + 1000 * rank)
+    T, H, E, I, k = inp["T"], inp["H"], inp["E"], inp["I"], inp["top_k"]
+    dt = layer.dtype_code(inp["w13"])
+    ws = layer.make_workspace(T, H, E, I, k, dt, dev)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    fwd = dict(w13_scale=inp["w13_scale"], w2_scale=inp["w2_scale"], out=out, workspace=ws)
+
+    def step(events=None):
+        layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                          stage_events=events, **fwd)
+
+    # warm-up (also yields the routing this batch produces)
+    dbg = {}
+    layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                      debug=dbg, **fwd)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    code, info = layer.get_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} info {info:#x} after warm-up")
+    counts = dbg["counts"].cpu().numpy()
+    e_act = int((counts > 0).sum())
+    esize = 1 if dt == 1 else 2
+    w13_bytes = e_act * 2 * I * H * esize
+    w2_bytes = e_act * H * I * esize
+    weight_bytes = w13_bytes + w2_bytes
+
+    from mixture_experts_layer_counts_b200.layer import N_STAGE_EVENTS, STAGES
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(N_STAGE_EVENTS)] for _ in range(args.steps)]
+    for row in evs:              # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    code, info = layer.get_status(ws)
+    if code != 0:
+        raise RuntimeError(f"device status {code} info {info:#x} in the timed region")
+    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
+    stage_ms = {STAGES[s]: sum(evs[i][s - 1].elapsed_time(evs[i][s]) for i in range(args.steps)) / args.steps
+                for s in range(1, N_STAGE_EVENTS)}
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms * 1e-3)
+
+    # end to end: pinned host hidden in, pinned host out, copies inside the timed region
+    hin = inp["hidden"].cpu().pin_memory()
+    hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(10, min(args.steps, 200))
+    e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(e2e_steps):
+        flush.zero_()
+        e_ev[i][0].record(stream)
+        layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k, hout, ws,
+                                 inp["w13_scale"], inp["w2_scale"])
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world)
+    e2e_value = world * T * e2e_steps / (e2e_ms * 1e-3)
+
+    peak, peak_kind = peaks()
+    w13_s = stage_ms["w13"] * 1e-3
+    achieved = w13_bytes / w13_s / 1e9
+    line = {
+        "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8-e4m3" if dt == 1 else "bf16", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: {describe(wl)}", "global_batch": world * T,
+                   "active_experts": e_act, "l2": "flushed (256 MiB write) between timed steps",
+                   "parallelism": f"dp{world} (independent decode batches)"},
+        "us_per_layer": 1e3 * ms_per_step,
+        "weight_bytes": weight_bytes,
+        "weight_gbs": weight_bytes / (ms_per_step * 1e-3) / 1e9,
+        "weight_gbs_frac_of_measured_hbm": weight_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
+        "weight_gbs_frac_of_8tbs": weight_bytes / (ms_per_step * 1e-3) / 8e12,
+        "stages_us": {k_: 1e3 * v for k_, v in stage_ms.items()},
+        "roofline": {"kernel": "grouped_gemm_kernel<swap-AB, w13>", "bound": "hbm", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": kernel_traffic(args.workload), "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": w13_bytes},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+                "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps},
+        "gpu_launches": launches_per_step(wl, T) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = host_copy(inp)
+        toks = list(range(min(CPU_BASELINE_TOKENS, T)))
+        secs = oracle_sample_seconds(host, wl, toks)
+        line["cpu_baseline"] = {"value": len(toks) / secs, "unit": "tokens/s", "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"fp64 oracle on tokens 0..{len(toks) - 1} of the batch "
+                                          f"(routing of all {T} tokens), {secs:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 5000; reference: 5)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default 20; reference: 1)")
+    ap.add_argument("--workload", default="decode", choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        # the fp64 oracle takes seconds per token: small defaults, one-token samples
+        args.steps = 5 if args.steps is None else args.steps
+        args.warmup = 1 if args.warmup is None else args.warmup
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        run_reference(args, wl, rank, world)
+        return
+    args.steps = 5000 if args.steps is None else args.steps
+    args.warmup = 20 if args.warmup is None else args.warmup
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, wl, rank, world, local)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
