@@ -67,7 +67,9 @@ typedef enum {
   MOE_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
   MOE_ERR_DEVICE_TIMEOUT = 5,     /* a bounded device-side wait expired */
   MOE_ERR_DEVICE_BOUNDS = 6,      /* an expert id outside [0, E) reached moe_align */
-  MOE_ERR_MISALIGNED = 7          /* a pointer is not 16-byte aligned */
+  MOE_ERR_MISALIGNED = 7,         /* a pointer is not 16-byte aligned */
+  MOE_ERR_EXCEEDS_STATIC_SCRATCH = 8  /* moe_route_static: T and E need more than its
+                                         fixed 8 MiB scratch */
 } moe_status_t;
 
 /* Optional outputs of moe_forward for checking and profiling; every field may
@@ -137,6 +139,28 @@ moe_status_t moe_route(const void *hidden, const void *router_w, const float *ro
 moe_status_t moe_align(const int32_t *topk_ids, int T, int E, int top_k, int32_t *counts,
                        int32_t *offsets, int32_t *perm, int32_t *inv_perm, void *workspace,
                        size_t workspace_bytes, void *stream);
+
+/* Router for callers that cannot allocate device memory.  (No counterpart in
+ * the pages: it is an interface of this library, not part of the method.)
+ * Same computation and outputs as moe_route, but with no workspace argument:
+ * its scratch is one 8 MiB array inside the library, fixed at build time.
+ * Meant for code that receives its input and output buffers from a host
+ * program but has no allocator of its own (a plug-in inside a runtime that
+ * owns all device memory, or a hot loop that must not allocate).
+ *   - Allocates nothing: no cudaMalloc / cudaFree, no library allocator.
+ *   - The array exists on every GPU that loads this library, until exit.
+ *   - Capacity: 20 * T * E + 4 * (2T + E) bytes plus alignment must fit in
+ *     8 MiB (about T * E <= 400,000, e.g. T = 2048 with E = 128); larger
+ *     shapes return MOE_ERR_EXCEEDS_STATIC_SCRATCH before anything runs.
+ *   - The first call on a device looks up the array's device address; make
+ *     that first call outside any stream capture.
+ *   - All calls share the array: calls that may overlap on the GPU (other
+ *     streams, other host threads) race and must be serialised by the caller.
+ *   - Device-side status words live in the array too and are cleared at the
+ *     start of every call; moe_get_status does not apply. */
+moe_status_t moe_route_static(const void *hidden, const void *router_w, const float *router_bias,
+                              int T, int H, int E, int top_k, int32_t *topk_ids, float *topk_w,
+                              void *stream);
 
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace since the last call (MOE_OK if none) and clears it.  *info_out

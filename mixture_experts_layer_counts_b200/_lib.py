@@ -18,12 +18,12 @@ MOE_DTYPE_FP8_E4M3 = 1
 STATUS = {
     0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED_SHAPE",
     3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_TIMEOUT",
-    6: "MOE_ERR_DEVICE_BOUNDS", 7: "MOE_ERR_MISALIGNED",
+    6: "MOE_ERR_DEVICE_BOUNDS", 7: "MOE_ERR_MISALIGNED", 8: "MOE_ERR_EXCEEDS_STATIC_SCRATCH",
 }
 
 # every symbol include/moe.h declares
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_forward", "moe_forward_hostio",
-           "moe_route", "moe_align", "moe_get_status", "moe_status_string")
+           "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static")
 
 
 class DebugOut(C.Structure):
@@ -63,6 +63,8 @@ def lib() -> C.CDLL:
         L.moe_forward_hostio.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, vp]
         L.moe_route.restype = i
         L.moe_route.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, sz, vp]
+        L.moe_route_static.restype = i
+        L.moe_route_static.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp]
         L.moe_align.restype = i
         L.moe_align.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, sz, vp]
         L.moe_get_status.restype = i

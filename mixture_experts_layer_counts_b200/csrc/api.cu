@@ -356,6 +356,7 @@ const char* moe_status_string(moe_status_t s) {
     case MOE_ERR_DEVICE_TIMEOUT: return "device wait timed out";
     case MOE_ERR_DEVICE_BOUNDS: return "expert id out of range";
     case MOE_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case MOE_ERR_EXCEEDS_STATIC_SCRATCH: return "shape exceeds the fixed static scratch";
   }
   return "unknown status";
 }
