@@ -1,12 +1,12 @@
 /*
  * moe.h -- C ABI of the B200 (sm_100a) fused Mixture-of-Experts layer.
  *
- * What it computes.  Fused MoE "combines token routing, data transfers and
- * expert computation into a single batched operation on the GPU" ("AWS
+ * What it computes.  Fused MoE is one batched GPU operation covering token
+ * routing, the movement of token data and the experts' arithmetic ("AWS
  * describes a fused MoE optimization for the NVIDIA Hopper architecture",
- * body) and fuses "scaling, matrix multiplication and expert aggregation"
- * ("AWS details MoE kernel fixes for SageMaker, upstreams them to vLLM",
- * paragraph on the Triton backend).  For each token t:
+ * body), with scaling, matrix products and the aggregation of expert outputs
+ * done in one pass ("AWS details MoE kernel fixes for SageMaker, upstreams
+ * them to vLLM", paragraph on the Triton backend).  For each token t:
  *   logits[e] = hidden[t] . router_w[e] (+ router_bias[e])
  *   p         = fp32 softmax over the E logits
  *   ids       = the top_k experts by logit, descending, exact ties -> lower id

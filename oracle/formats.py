@@ -14,8 +14,9 @@ Formats:
   3 mantissa bits, no infinities, NaN only at S.1111.111, largest finite 448.
   Encoding here is RNE followed by saturation to +-448 ("satfinite"), the
   convention the fused-MoE FP8 path uses for both activations and the
-  intermediate (the pages call the scheme "tensor-quantized"; they do not
-  spell out the rounding, so RNE + saturation is the reading taken).
+  intermediate (the pages only say the FP8 models use one scale per tensor;
+  they do not spell out the rounding, so RNE + saturation is the reading
+  taken).
 
 Every function works element-wise on numpy arrays and is vectorised only with
 plain numpy primitives (frexp, rint, where), so each line can be checked

@@ -5,13 +5,13 @@ by ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
 ``--impl reference`` legs of ``bench.py``.  The product path (the CUDA
 library and its Python binding) never touches it and shares no code with it.
 
-What the layer computes.  The pages describe fused MoE only in words: it
-"combines token routing, data transfers and expert computation into a single
-batched operation" ("AWS describes a fused MoE optimization for the NVIDIA
-Hopper architecture", body) and fuses "scaling, matrix multiplication and
-expert aggregation" ("AWS details MoE kernel fixes...", body paragraph on the
-Triton backend).  The step-by-step definition followed here is the plain
-gated-MLP MoE layer:
+What the layer computes.  The pages describe fused MoE only in words: one
+batched GPU operation that does the routing of tokens, the movement of their
+data and the experts' arithmetic ("AWS describes a fused MoE optimization for
+the NVIDIA Hopper architecture", body), with the scaling, the matrix products
+and the aggregation of expert outputs done in one pass ("AWS details MoE
+kernel fixes...", body paragraph on the Triton backend).  The step-by-step
+definition followed here is the plain gated-MLP MoE layer:
 
   R0  decode the given bf16 / E4M3 bytes exactly; dequantised weight =
       code value * per-expert fp32 scale.
