@@ -261,28 +261,72 @@ def run_ours(args, wl, rank, world, local):
 
     from mixture_experts_layer_counts_b200.layer import N_STAGE_EVENTS, STAGES
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(N_STAGE_EVENTS)] for _ in range(args.steps)]
-    for row in evs:              # torch creates the CUDA event on first record
-        for ev in row:
+    def new_events(n):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for ev in evs:           # torch creates the CUDA event on first record
             ev.record(stream)
+        return evs
+
+    # The timed step is one replay of a CUDA graph holding one layer call, the
+    # way a decode engine runs it (kernels chained by programmatic dependent
+    # launch).  Start/end events are recorded on the stream around each
+    # replay; the L2 flush sits between steps, outside the events.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        flush.zero_()
+        graph.replay()
+    tev = [new_events(2) for _ in range(args.steps)]
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for i in range(args.steps):
             flush.zero_()
-            step(evs[i])
+            tev[i][0].record(stream)
+            graph.replay()
+            tev[i][1].record(stream)
         torch.cuda.synchronize()
     barrier(world)
     code, info = layer.get_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} info {info:#x} in the timed region")
-    step_ms = [evs[i][0].elapsed_time(evs[i][-1]) for i in range(args.steps)]
-    stage_ms = {STAGES[s]: sum(evs[i][s - 1].elapsed_time(evs[i][s]) for i in range(args.steps)) / args.steps
-                for s in range(1, N_STAGE_EVENTS)}
+    step_ms = [a_.elapsed_time(b_) for a_, b_ in tev]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     value = world * T * args.steps / (total_ms * 1e-3)
+    del graph
+
+    # Per-kernel breakdown: the same graph with the library's 8 stage events
+    # recorded inside it (each event node costs ~2-3 us, so these stage times
+    # are upper bounds and their sum exceeds the step time above).
+    gev = new_events(N_STAGE_EVENTS)
+    torch.cuda.synchronize()
+    igraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(igraph):
+        step(gev)
+    n_stage = min(args.steps, 1000)
+    stage_sum = [0.0] * (N_STAGE_EVENTS - 1)
+    for i in range(n_stage + 3):
+        flush.zero_()
+        igraph.replay()
+        gev[-1].synchronize()
+        if i >= 3:
+            for s in range(1, N_STAGE_EVENTS):
+                stage_sum[s - 1] += gev[s - 1].elapsed_time(gev[s])
+    stage_ms = {STAGES[s]: stage_sum[s - 1] / n_stage for s in range(1, N_STAGE_EVENTS)}
+    del igraph
+
+    # the same step launched directly (no graph): host launch gaps included
+    n_direct = min(args.steps, 500)
+    dev_ = [new_events(N_STAGE_EVENTS) for _ in range(n_direct)]
+    torch.cuda.synchronize()
+    for i in range(n_direct):
+        flush.zero_()
+        step(dev_[i])
+    torch.cuda.synchronize()
+    direct_ms = max_over_ranks(sum(e[0].elapsed_time(e[-1]) for e in dev_), world) / n_direct
 
     # end to end: pinned host hidden in, pinned host out, copies inside the timed region
     hin = inp["hidden"].cpu().pin_memory()
@@ -314,6 +358,10 @@ def run_ours(args, wl, rank, world, local):
                    "active_experts": e_act, "l2": "flushed (256 MiB write) between timed steps",
                    "parallelism": f"dp{world} (independent decode batches)"},
         "us_per_layer": 1e3 * ms_per_step,
+        "us_per_layer_p50": 1e3 * statistics.median(step_ms),
+        "us_per_layer_direct_launch": 1e3 * direct_ms,
+        "timing": "per step: device time of one CUDA-graph replay of moe_forward (events on the "
+                  "stream around the replay); stages_us from a separate instrumented graph",
         "weight_bytes": weight_bytes,
         "weight_gbs": weight_bytes / (ms_per_step * 1e-3) / 1e9,
         "weight_gbs_frac_of_measured_hbm": weight_bytes / (ms_per_step * 1e-3) / 1e9 / peak,

@@ -60,7 +60,11 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   const int A = a.T * a.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
+  pdl_wait();
+  pdl_launch_next();
   for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  if (a.gemm_flags != nullptr)
+    for (int i = threadIdx.x; i < a.n_gemm_flags; i += blockDim.x) a.gemm_flags[i] = 0;
   __syncthreads();
 
   const int per = (A + 31) / 32;
@@ -114,12 +118,12 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
     __syncwarp();
   }
 
-  // tile schedule: swap-AB chunks of <= kSwapMaxTokens tokens for experts
+  // tile schedule: swap-AB chunks of <= swap_chunk tokens for experts
   // with count <= swap_max_count, normal-orientation tiles of kNormalTokens
   // tokens for the rest.
   const bool ex = threadIdx.x < E && c > 0;
   const bool sw = ex && c <= a.swap_max_count;
-  const int nsw = sw ? (c + kSwapMaxTokens - 1) / kSwapMaxTokens : 0;
+  const int nsw = sw ? (c + a.swap_chunk - 1) / a.swap_chunk : 0;
   const int nno = (ex && !sw) ? (c + kNormalTokens - 1) / kNormalTokens : 0;
   const int osw = block_exclusive_scan(nsw, tmp32, &total);
   const int tsw = total;
@@ -127,8 +131,8 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   const int ono = block_exclusive_scan(nno, tmp32, &total);
   const int tno = total;
   for (int i = 0; i < nsw; ++i) {
-    const int n0 = i * kSwapMaxTokens;
-    a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(kSwapMaxTokens, c - n0), 0);
+    const int n0 = i * a.swap_chunk;
+    a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(a.swap_chunk, c - n0), 0);
   }
   for (int i = 0; i < nno; ++i) {
     const int n0 = i * kNormalTokens;
@@ -158,10 +162,9 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
 
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t st) {
   const size_t smem = static_cast<size_t>(32) * a.E * sizeof(int);
-  cudaFuncSetAttribute(align_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       static_cast<int>(smem));
-  align_kernel<<<1, 1024, smem, st>>>(a);
-  return cudaGetLastError();
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(align_kernel), static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  return launch_pdl(align_kernel, dim3(1), dim3(1024), smem, st, a);
 }
 
 }  // namespace moe

@@ -13,6 +13,33 @@
 #include "moe.h"
 
 namespace moe {
+
+cudaError_t set_smem_limit_once(const void* kernel, int bytes) {
+  struct Entry {
+    const void* kernel;
+    int device;
+    int bytes;
+  };
+  static std::mutex mu;
+  static Entry table[256];
+  static int n = 0;
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n; ++i)
+    if (table[i].kernel == kernel && table[i].device == dev && table[i].bytes >= bytes) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err != cudaSuccess) return err;
+  for (int i = 0; i < n; ++i)
+    if (table[i].kernel == kernel && table[i].device == dev) {
+      table[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (n < 256) table[n++] = Entry{kernel, dev, bytes};
+  return cudaSuccess;
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -101,9 +128,16 @@ moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE
     if (s_ != MOE_OK) return s_;       \
   } while (0)
 
+// Stage events: inside a stream capture a plain record would only be a
+// dependency marker of the graph, so record "external" event nodes there.
 void record(moe_debug_out_t* dbg, int i, cudaStream_t st) {
-  if (dbg && dbg->stage_events && dbg->stage_events[i])
-    cudaEventRecord(static_cast<cudaEvent_t>(dbg->stage_events[i]), st);
+  if (!(dbg && dbg->stage_events && dbg->stage_events[i])) return;
+  cudaEvent_t ev = static_cast<cudaEvent_t>(dbg->stage_events[i]);
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
 }
 
 moe_status_t forward_impl(const void* hidden, const void* router_w, const float* router_bias,
@@ -161,7 +195,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
-               tau, fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr};
+               tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
+               at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots};
   MOE_TRY(cuda_status(launch_align(aa, st)));
   record(dbg, 2, st);
 
@@ -169,7 +204,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                                     A, k, H, fp8, hdr, xperm, st)));
   record(dbg, 3, st);
 
-  const int grid = device_sm_count() < kMaxGrid ? device_sm_count() : kMaxGrid;
+  const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;
+  int* flags = at<int>(ws, L.gemm_flags);   // one kMaxSlots array per GEMM launch
   GemmArgs g13{};
   g13.katoms = H * (fp8 ? 1 : 2) / kAtomBytes;
   g13.w_rows_per_expert = 2 * I;
@@ -182,6 +218,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g13.wscale = w13_scale;
   g13.act_scale = hdr + kHdrScaleS1;
   g13.hdr = hdr;
+  g13.partials = at<float>(ws, L.partials);
   float* amax_cta = at<float>(ws, L.amax_cta);
   if (any_swap) {
     GemmArgs g = g13;
@@ -189,6 +226,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.nchunks = hdr + kHdrChunksSwap;
     g.mtiles = I / kTileM;
     g.amax_cta = amax_cta;
+    g.flags = flags + 0 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW13, fp8, tw13s, txs, g, grid, st)));
   }
   if (any_normal) {
@@ -197,6 +235,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.nchunks = hdr + kHdrChunksNormal;
     g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
     g.amax_cta = amax_cta + (any_swap ? grid : 0);
+    g.flags = flags + 1 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
   }
   record(dbg, 4, st);
@@ -221,6 +260,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.chunks = at<int4>(ws, L.chunks_swap);
     g.nchunks = hdr + kHdrChunksSwap;
     g.mtiles = H / kTileM;
+    g.flags = flags + 2 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, fp8, tw2s, tis, g, grid, st)));
   }
   if (any_normal) {
@@ -228,6 +268,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.chunks = at<int4>(ws, L.chunks_normal);
     g.nchunks = hdr + kHdrChunksNormal;
     g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
+    g.flags = flags + 3 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
   }
   record(dbg, 6, st);
@@ -323,11 +364,12 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!topk_ids || !counts || !offsets || !perm || !inv_perm || !workspace) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(T, 128, E, 128, top_k, false);
-  if (workspace_bytes < L.chunks_normal + static_cast<size_t>(L.max_chunks_normal) * 16)
+  if (workspace_bytes < L.gemm_flags + static_cast<size_t>(kGemmLaunches) * kMaxSlots * 4)
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   AlignArgs aa{topk_ids, T, E, top_k, counts, offsets, perm, inv_perm,
                at<int4>(workspace, L.chunks_swap), at<int4>(workspace, L.chunks_normal),
-               swap_threshold(), nullptr, at<uint32_t>(workspace, L.header)};
+               swap_threshold(), gemm_swap_chunk(), nullptr, at<uint32_t>(workspace, L.header),
+               at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots};
   return cuda_status(launch_align(aa, static_cast<cudaStream_t>(stream)));
 }
 

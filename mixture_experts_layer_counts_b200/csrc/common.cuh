@@ -35,6 +35,9 @@ constexpr int kNormalTokens = 128;     // token rows per tile in normal orientat
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxGrid = 1024;          // persistent grids never exceed this
+constexpr int kMaxSlots = 160;          // GEMM CTAs per launch (>= the SM count of a B200)
+constexpr int kPartialSlotFloats = 32768;   // fp32 partial tile of one GEMM CTA (128 KB)
+constexpr int kGemmLaunches = 4;        // {w13, w2} x {swap-AB, normal}: one flag array each
 
 // Header words at the start of the workspace (uint32 units).
 constexpr int kHdrStatus = 0;          // first device error code (sticky)
@@ -56,7 +59,7 @@ __device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, u
 // Byte offsets of every region of the caller-provided workspace.
 struct Layout {
   size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand;
-  size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal;
+  size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, gemm_flags, partials;
   size_t xperm, inter, h32, ysc, staging_in, staging_out, total;
   int max_chunks_swap, max_chunks_normal;
 };
@@ -85,10 +88,12 @@ inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   L.offsets = take(static_cast<size_t>(E + 1) * 4);
   L.perm = take(A * 4);
   L.inv_perm = take(A * 4);
-  L.max_chunks_swap = static_cast<int>(E + A / kSwapMaxTokens + 1);
+  L.max_chunks_swap = static_cast<int>(E + A / 16 + 1);   // swap chunks hold >= 16 tokens
   L.max_chunks_normal = static_cast<int>(E + A / kNormalTokens + 1);
   L.chunks_swap = take(static_cast<size_t>(L.max_chunks_swap) * 16);
   L.chunks_normal = take(static_cast<size_t>(L.max_chunks_normal) * 16);
+  L.gemm_flags = take(static_cast<size_t>(kGemmLaunches) * kMaxSlots * 4);
+  L.partials = take(static_cast<size_t>(kMaxSlots) * kPartialSlotFloats * 4);
   const size_t eb = fp8 ? 1 : 2;
   L.xperm = take(A * H * eb);
   L.inter = take(A * I * eb);

@@ -34,6 +34,8 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 
 __global__ void gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm,
                               int A, int k, int vpr, uint4* __restrict__ xperm) {
+  pdl_wait();
+  pdl_launch_next();
   const int T = A / k;
   const size_t n = static_cast<size_t>(A) * vpr;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
@@ -48,6 +50,8 @@ __global__ void gather_kernel(const uint4* __restrict__ hidden, const int32_t* _
 __global__ void gather_quant_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm,
                                     int A, int k, int vpr, const uint32_t* __restrict__ hdr,
                                     uint2* __restrict__ xq) {
+  pdl_wait();
+  pdl_launch_next();
   const int T = A / k;
   const float s1 = __uint_as_float(hdr[kHdrScaleS1]);
   const size_t n = static_cast<size_t>(A) * vpr;
@@ -72,6 +76,8 @@ __global__ void gather_quant_kernel(const uint4* __restrict__ hidden, const int3
 __global__ void requant_kernel(const float4* __restrict__ h32, const float* __restrict__ amax_cta,
                                int n_cta, size_t n4, uint32_t* __restrict__ hdr,
                                uint32_t* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_next();
   __shared__ float s_scale;
   if (threadIdx.x < 32) {
     float m = 0.f;
@@ -96,19 +102,34 @@ __global__ void requant_kernel(const float4* __restrict__ h32, const float* __re
 
 __global__ void combine_kernel(const float4* __restrict__ ysc, int T, int k, int h4,
                                uint2* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_next();
   const size_t n = static_cast<size_t>(T) * h4;
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int t = static_cast<int>(i / h4);
     const int c = static_cast<int>(i - static_cast<size_t>(t) * h4);
     const float4* src = ysc + static_cast<size_t>(t) * k * h4 + c;
-    float4 acc = src[0];
-    for (int j = 1; j < k; ++j) {
-      const float4 y = src[static_cast<size_t>(j) * h4];
-      acc.x += y.x;
-      acc.y += y.y;
-      acc.z += y.z;
-      acc.w += y.w;
+    // loads of up to 8 slots are issued together; the sum stays in slot order
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      float4 y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < k) y[u] = __ldcg(src + static_cast<size_t>(j0 + u) * h4);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u < k) {
+          if (j0 + u == 0) {
+            acc = y[u];
+          } else {
+            acc.x += y[u].x;
+            acc.y += y[u].y;
+            acc.z += y[u].z;
+            acc.w += y[u].w;
+          }
+        }
+      }
     }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
     __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
@@ -122,21 +143,19 @@ cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int 
   const size_t n = static_cast<size_t>(A) * vpr;
   const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
   if (fp8)
-    gather_quant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(hidden), perm, A, k,
-                                              vpr, hdr, reinterpret_cast<uint2*>(xperm));
-  else
-    gather_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(hidden), perm, A, k, vpr,
-                                        reinterpret_cast<uint4*>(xperm));
-  return cudaGetLastError();
+    return launch_pdl(gather_quant_kernel, dim3(grid), dim3(256), 0, st,
+                      reinterpret_cast<const uint4*>(hidden), perm, A, k, vpr, hdr,
+                      reinterpret_cast<uint2*>(xperm));
+  return launch_pdl(gather_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const uint4*>(hidden),
+                    perm, A, k, vpr, reinterpret_cast<uint4*>(xperm));
 }
 
 cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
                            uint32_t* hdr, uint8_t* inter, cudaStream_t st) {
   const size_t n4 = count / 4;
   const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, static_cast<size_t>(sm_count()) * 8));
-  requant_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(h32), amax_cta, n_cta, n4,
-                                       hdr, reinterpret_cast<uint32_t*>(inter));
-  return cudaGetLastError();
+  return launch_pdl(requant_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(h32),
+                    amax_cta, n_cta, n4, hdr, reinterpret_cast<uint32_t*>(inter));
 }
 
 cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
@@ -144,9 +163,8 @@ cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16*
   const int h4 = H / 4;
   const size_t n = static_cast<size_t>(T) * h4;
   const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
-  combine_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const float4*>(ysc), T, k, h4,
-                                       reinterpret_cast<uint2*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(ysc), T,
+                    k, h4, reinterpret_cast<uint2*>(out));
 }
 
 }  // namespace moe

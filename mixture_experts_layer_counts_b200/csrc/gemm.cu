@@ -23,6 +23,16 @@
 //          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), which
 //          the combine pass sums in slot order: deterministic, no atomics.
 //
+// Work split (balanced over the persistent CTAs).  A "unit" is one output
+// tile (token chunk x weight-row tile) and needs `katoms` K atoms.  The
+// nunits * katoms atoms are cut into G equal contiguous ranges, one per CTA,
+// so every SM streams the same number of weight bytes whatever the number of
+// active experts.  A unit cut by a range boundary is finished by the CTA that
+// holds its first atoms (the "head", whose range ends there, so it reaches
+// that unit last): the CTAs holding the later atoms write their fp32 partial
+// accumulators to their own slot and raise a flag; the head adds the partials
+// in K order and runs the epilogue.  Fixed order, no atomics on data.
+//
 // Pipeline per CTA (192 threads):
 //   warp 0 lane 0  TMA producer: STAGES-deep ring of {A, B} tiles, 128-byte
 //                  K atoms in the 128B-swizzle layout, mbarrier complete_tx.
@@ -31,10 +41,12 @@
 //                  final commit hands the TMEM buffer to the epilogue.
 //   warps 2..5     epilogue: tcgen05.ld 32 lanes x 16 columns per warp
 //                  (warp w reads TMEM lanes 32*(w%4)..+31), math, stores.
-// Two TMEM accumulator buffers, so the epilogue of one tile overlaps the
+// Two TMEM accumulator buffers, so the epilogue of one segment overlaps the
 // mainloop of the next.  Every wait is bounded (see mbar_wait).
 #include <cuda.h>
 #include <cuda_bf16.h>
+
+#include <cstdlib>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -42,32 +54,100 @@
 
 namespace moe {
 
-template <Orient O, Proj P, bool FP8>
+// KA = K atoms per pipeline stage (each weight row then contributes KA*128
+// contiguous bytes per stage); BNT = largest token chunk of the swap-AB form.
+template <Orient O, Proj P, bool FP8, int KA, int BNT>
 struct Cfg {
   static constexpr bool kSwap = O == Orient::kSwap;
   static constexpr bool kDual = P == Proj::kW13;
-  static constexpr int kBN = kSwap ? kSwapMaxTokens : (kDual ? 128 : 256);   // max N
+  static constexpr int kBN = kSwap ? BNT : (kDual ? 128 : 256);   // max N
   static constexpr int kATile = kTileM * kAtomBytes;
   static constexpr int kBTile = kBN * kAtomBytes;
   static constexpr int kNumA = (kSwap && kDual) ? 2 : 1;
   static constexpr int kNumB = (!kSwap && kDual) ? 2 : 1;
-  static constexpr int kStageBytes = kNumA * kATile + kNumB * kBTile;
-  static constexpr int kStages = (kSwap && kDual) ? 5 : (kSwap ? 8 : 4);
-  static constexpr int kAccCols = (kDual ? 2 : 1) * kBN;       // per TMEM buffer
+  static constexpr int kAtomSet = kNumA * kATile + kNumB * kBTile;   // one K atom of every operand
+  static constexpr int kStageBytes = KA * kAtomSet;
+  static constexpr int kStagesFit = (232448 - 1280) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kNumAcc = kDual ? 2 : 1;
+  static constexpr int kAccCols = kNumAcc * kBN;               // per TMEM buffer
   static constexpr int kTmemCols = 2 * kAccCols;               // 128, 256 or 512
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr int kAtomElems = FP8 ? 128 : 64;
-  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM columns");
+  static constexpr int kSlotFloats = kNumAcc * kTileM * kBN;   // one CTA's partial tile
+  static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
+                "TMEM allocations are powers of two from 32 to 512 columns");
   static_assert(kSmemBytes <= 232448, "shared memory");
+  static_assert(kSlotFloats <= kPartialSlotFloats, "partial slot");
+  static_assert(kStages >= 2, "pipeline depth");
 };
 
 constexpr int kThreads = 192;
+constexpr int kMinAtomsPerCta = 8;   // below this, fewer CTAs share the work
 
-template <Orient O, Proj P, bool FP8>
+// Contiguous atom range of CTA c out of G over W atoms, and the CTA owning atom a.
+__device__ __forceinline__ long long range_begin(long long W, int G, int c) {
+  return static_cast<long long>(c) * W / G;
+}
+__device__ __forceinline__ int atom_owner(long long a, long long W, int G) {
+  return static_cast<int>(((a + 1) * G - 1) / W);
+}
+
+// Walks one CTA's atom range as (unit, first atom, end atom) segments.
+struct Segments {
+  long long a, a1;
+  int katoms;
+  __device__ bool next(int& u, int& kb0, int& kb1) {
+    if (a >= a1) return false;
+    u = static_cast<int>(a / katoms);
+    kb0 = static_cast<int>(a - static_cast<long long>(u) * katoms);
+    const long long left = a1 - a;
+    kb1 = left < katoms - kb0 ? kb0 + static_cast<int>(left) : katoms;
+    a += kb1 - kb0;
+    return true;
+  }
+};
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void epilogue_bar() {   // the 4 epilogue warps only
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait for a neighbour CTA's partial-tile flag.
+__device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, uint32_t* status) {
+  if (ld_acquire(flag) != 0) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire(flag) != 0) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        report_status(status, MOE_DEVICE_TIMEOUT, kSiteGridBarrier);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+template <Orient O, Proj P, bool FP8, int KA, int BNT>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
-  using C = Cfg<O, P, FP8>;
+  using C = Cfg<O, P, FP8, KA, BNT>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base for the swizzled tiles
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -85,6 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // prologue (overlaps the previous kernel's tail under programmatic launch)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -96,6 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    red[0] = red[1] = red[2] = red[3] = 0.f;
     fence_barrier_init();
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
@@ -109,9 +191,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int nunits = static_cast<int>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
+  grid_dependency_wait();   // the tile schedule and activations come from earlier kernels
+  grid_dependents_launch();
 
-  if (warp == 0 && lane == 0) {
+  const long long nunits =
+      static_cast<long long>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
+  const int ksteps = a.katoms / KA;   // pipeline stages per unit
+  const long long W = nunits * ksteps;
+  int G = static_cast<int>(W / kMinAtomsPerCta);
+  G = G < 1 ? 1 : (G > static_cast<int>(gridDim.x) ? static_cast<int>(gridDim.x) : G);
+  const bool active = W > 0 && static_cast<int>(blockIdx.x) < G;
+  const long long my_a0 = active ? range_begin(W, G, blockIdx.x) : 0;
+  const long long my_a1 = active ? range_begin(W, G, blockIdx.x + 1) : 0;
+
+  if (warp == 0 && lane == 0 && active) {
     // ------------------------------------------------------- TMA producer --
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_x = l2_policy_evict_last();
@@ -119,7 +212,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per-stage bookkeeping for the abort drain
     bool ok = true;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x) {
+    Segments seg{my_a0, my_a1, ksteps};
+    int u, kb0, kb1;
+    while (ok && seg.next(u, kb0, kb1)) {
       const int4 ch = a.chunks[u / a.mtiles];
       const int mt = u % a.mtiles;
       const int e = ch.x, p0 = ch.y, nv = ch.z;
@@ -129,13 +224,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (C::kSwap) {
         const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
         nbox = nvpad / kTokenBox;
-        bytes = C::kNumA * C::kATile + nvpad * kAtomBytes;
+        bytes = KA * (C::kNumA * C::kATile + nvpad * kAtomBytes);
         wrow0 = e * a.w_rows_per_expert + mt * kTileM;
       } else {
         bytes = C::kStageBytes;
         wrow0 = e * a.w_rows_per_expert + mt * C::kBN;
       }
-      for (int kb = 0; kb < a.katoms; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty)) {
           ok = false;
           break;
@@ -144,18 +239,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[stage], bytes);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        const int kc = kb * C::kAtomElems;
-        if constexpr (C::kSwap) {
-          tma_load_2d(st, &tm_w, &full[stage], kc, wrow0, pol_w);
-          if constexpr (C::kDual) tma_load_2d(st + C::kATile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
-          uint8_t* sb = st + C::kNumA * C::kATile;
-          for (int q = 0; q < nbox; ++q)
-            tma_load_2d(sb + q * kTokenBox * kAtomBytes, &tm_x, &full[stage], kc, p0 + q * kTokenBox, pol_x);
-        } else {
-          tma_load_2d(st, &tm_x, &full[stage], kc, p0, pol_x);
-          tma_load_2d(st + C::kATile, &tm_w, &full[stage], kc, wrow0, pol_w);
-          if constexpr (C::kDual)
-            tma_load_2d(st + C::kATile + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+#pragma unroll
+        for (int ka = 0; ka < KA; ++ka) {
+          uint8_t* sa = st + ka * C::kAtomSet;
+          const int kc = (kb * KA + ka) * C::kAtomElems;
+          if constexpr (C::kSwap) {
+            tma_load_2d(sa, &tm_w, &full[stage], kc, wrow0, pol_w);
+            if constexpr (C::kDual) tma_load_2d(sa + C::kATile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+            uint8_t* sb = sa + C::kNumA * C::kATile;
+            for (int q = 0; q < nbox; ++q)
+              tma_load_2d(sb + q * kTokenBox * kAtomBytes, &tm_x, &full[stage], kc, p0 + q * kTokenBox, pol_x);
+          } else {
+            tma_load_2d(sa, &tm_x, &full[stage], kc, p0, pol_x);
+            tma_load_2d(sa + C::kATile, &tm_w, &full[stage], kc, wrow0, pol_w);
+            if constexpr (C::kDual)
+              tma_load_2d(sa + C::kATile + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+          }
         }
         if (++stage == C::kStages) {
           stage = 0;
@@ -171,16 +270,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait(&full[s], (armed_parity >> s) & 1u, reinterpret_cast<volatile int*>(&dummy),
                     a.hdr, kSiteDrainTma);
     }
-  } else if (warp == 1 && lane == 0) {
+  } else if (warp == 1 && lane == 0 && active) {
     // ---------------------------------------------------------- MMA issuer --
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
     bool ok = true;
     bool issued = false;
-    for (int u = blockIdx.x; u < nunits && ok; u += gridDim.x, ++it) {
+    Segments seg{my_a0, my_a1, ksteps};
+    int u, kb0, kb1;
+    while (ok && seg.next(u, kb0, kb1)) {
       const int buf = it & 1;
       const uint32_t accph = (it >> 1) & 1;
+      ++it;
       if (!mbar_wait(&acc_empty[buf], accph ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty)) {
         ok = false;
         break;
@@ -196,16 +298,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc = idesc_f32acc(FP8 ? 0u : 1u, kTileM, static_cast<uint32_t>(n));
       const uint32_t d0 = tmem_base + buf * C::kAccCols;
       const uint32_t d1 = d0 + C::kBN;
-      for (int kb = 0; kb < a.katoms; ++kb) {
+      for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag, a.hdr, kSiteMmaFull)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(tiles + stage * C::kStageBytes);
 #pragma unroll
-        for (int kk = 0; kk < kAtomBytes / 32; ++kk) {
-          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+        for (int kq = 0; kq < KA * (kAtomBytes / 32); ++kq) {
+          const int ka = kq / (kAtomBytes / 32), kk = kq % (kAtomBytes / 32);
+          const uint32_t st = smem_u32(tiles + stage * C::kStageBytes + ka * C::kAtomSet);
+          const uint32_t acc = (kb > kb0 || kq > 0) ? 1u : 0u;
           const uint32_t off = kk * 32;
           if constexpr (C::kSwap) {
             const uint32_t sb = st + C::kNumA * C::kATile;
@@ -233,35 +336,92 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(drain);
       mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), a.hdr, kSiteDrainMma);
     }
-  } else if (warp >= 2) {
+  } else if (warp >= 2 && active) {
     // ------------------------------------------------------------ epilogue --
     const int q = warp & 3;               // TMEM lane quadrant of this warp
     const int row = q * 32 + lane;        // accumulator row held by this thread
     float amax = 0.f;
     int it = 0;
-    for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++it) {
+    Segments seg{my_a0, my_a1, ksteps};
+    int u, kb0, kb1;
+    while (seg.next(u, kb0, kb1)) {
       const int buf = it & 1;
       const uint32_t accph = (it >> 1) & 1;
+      ++it;
       if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull)) break;
       tc_fence_after();
       const int4 ch = a.chunks[u / a.mtiles];
       const int mt = u % a.mtiles;
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
+      const int ncols = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox * kTokenBox : C::kBN;
+
+      if (kb0 > 0) {
+        // ---- later piece of a split unit: hand the raw accumulator over ----
+        float* slot = a.partials + static_cast<size_t>(blockIdx.x) * kPartialSlotFloats;
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float v[C::kNumAcc][16];
+          if constexpr (C::kDual)
+            tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, v[0], v[1]);
+          else
+            tmem_ld16_wait(tbase + c0, v[0]);
+#pragma unroll
+          for (int ac = 0; ac < C::kNumAcc; ++ac) {
+            float4* dst = reinterpret_cast<float4*>(slot + (static_cast<size_t>(ac) * kTileM + row) * C::kBN + c0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              __stcg(dst + j, make_float4(v[ac][4 * j], v[ac][4 * j + 1], v[ac][4 * j + 2], v[ac][4 * j + 3]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&acc_empty[buf]);
+        __threadfence();
+        epilogue_bar();
+        if (row == 0) st_release(a.flags + blockIdx.x, 1);
+        continue;
+      }
+
+      // ---- first atoms of the unit: collect the later pieces, then finish ----
+      int last = blockIdx.x;
+      if (kb1 < ksteps) {
+        const long long unit_end = (static_cast<long long>(u) + 1) * ksteps;
+        last = atom_owner(unit_end - 1, W, G);
+        bool ok = true;
+        for (int c2 = blockIdx.x + 1; c2 <= last && ok; ++c2) ok = wait_flag(a.flags + c2, abort_flag, a.hdr);
+        if (!ok) break;
+      }
+      auto add_partials = [&](float (&v)[C::kNumAcc][16], int c0) {
+        for (int c2 = blockIdx.x + 1; c2 <= last; ++c2) {
+          const float* slot = a.partials + static_cast<size_t>(c2) * kPartialSlotFloats;
+#pragma unroll
+          for (int ac = 0; ac < C::kNumAcc; ++ac) {
+            const float4* src = reinterpret_cast<const float4*>(slot + (static_cast<size_t>(ac) * kTileM + row) * C::kBN + c0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 p = __ldcg(src + j);
+              v[ac][4 * j] += p.x;
+              v[ac][4 * j + 1] += p.y;
+              v[ac][4 * j + 2] += p.z;
+              v[ac][4 * j + 3] += p.w;
+            }
+          }
+        }
+      };
+
       float scale = 1.f;
       if constexpr (FP8) scale = a.wscale[e] * __uint_as_float(*a.act_scale);
 
       if constexpr (C::kSwap && C::kDual) {
-        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
         const int irow = mt * kTileM + row;
-        for (int c0 = 0; c0 < nvpad; c0 += 16) {
-          float g[16], uu[16];
-          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, g, uu);
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float v[2][16];
+          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, v[0], v[1]);
+          add_partials(v, c0);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
             if (n < nv) {
-              const float gg = g[j] * scale, uv = uu[j] * scale;
+              const float gg = v[0][j] * scale, uv = v[1][j] * scale;
               const float h = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
               const size_t o = static_cast<size_t>(p0 + n) * a.ld_out + irow;
               if constexpr (FP8) {
@@ -274,18 +434,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if constexpr (C::kSwap) {
-        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
         const int hrow = mt * kTileM + row;
-        for (int c0 = 0; c0 < nvpad; c0 += 16) {
-          float y[16];
-          tmem_ld16_wait(tbase + c0, y);
+        for (int c0 = 0; c0 < ncols; c0 += 16) {
+          float v[1][16];
+          tmem_ld16_wait(tbase + c0, v[0]);
+          add_partials(v, c0);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = c0 + j;
             const int f = n < nv ? a.perm[p0 + n] : -1;
             if (f >= 0 && f < a.num_assign) {
               const float wt = a.topk_w[f];
-              static_cast<float*>(a.out)[static_cast<size_t>(f) * a.ld_out + hrow] = y[j] * scale * wt;
+              static_cast<float*>(a.out)[static_cast<size_t>(f) * a.ld_out + hrow] = v[0][j] * scale * wt;
             }
           }
         }
@@ -294,13 +454,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int p = p0 + row;
         const int i0 = mt * C::kBN;
         for (int c0 = 0; c0 < C::kBN; c0 += 16) {
-          float g[16], uu[16];
-          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, g, uu);
+          float v[2][16];
+          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, v[0], v[1]);
+          add_partials(v, c0);
           if (valid) {
             float h[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-              const float gg = g[j] * scale, uv = uu[j] * scale;
+              const float gg = v[0][j] * scale, uv = v[1][j] * scale;
               h[j] = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
             }
             const size_t o = static_cast<size_t>(p) * a.ld_out + i0 + c0;
@@ -333,14 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (valid) wt = a.topk_w[f] * scale;
         const int h0 = mt * C::kBN;
         for (int c0 = 0; c0 < C::kBN; c0 += 16) {
-          float y[16];
-          tmem_ld16_wait(tbase + c0, y);
+          float v[1][16];
+          tmem_ld16_wait(tbase + c0, v[0]);
+          add_partials(v, c0);
           if (valid) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
                                                     static_cast<size_t>(f) * a.ld_out + h0 + c0);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(y[4 * j] * wt, y[4 * j + 1] * wt, y[4 * j + 2] * wt, y[4 * j + 3] * wt);
+              dst[j] = make_float4(v[0][4 * j] * wt, v[0][4 * j + 1] * wt, v[0][4 * j + 2] * wt,
+                                   v[0][4 * j + 3] * wt);
           }
         }
       }
@@ -357,38 +520,58 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if constexpr (FP8 && Cfg<O, P, FP8>::kDual) {
+  if constexpr (FP8 && C::kDual) {
+    // every CTA of the grid writes its slot (0 when it had no work)
     if (threadIdx.x == 0)
       a.amax_cta[blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
   }
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
-template <Orient O, Proj P, bool FP8>
+template <Orient O, Proj P, bool FP8, int KA, int BNT>
 static cudaError_t launch_one(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
                               int grid, cudaStream_t st) {
-  using C = Cfg<O, P, FP8>;
-  auto kern = grouped_gemm_kernel<O, P, FP8>;
-  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  using C = Cfg<O, P, FP8, KA, BNT>;
+  auto kern = grouped_gemm_kernel<O, P, FP8, KA, BNT>;
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
-  kern<<<grid, kThreads, C::kSmemBytes, st>>>(tw, tx, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, st, tw, tx, a);
+}
+
+// Swap-AB pipeline shape: K atoms per stage (MOE_SWAP_KA=1|2, read once).
+static int swap_ka() {
+  static int v = 0;
+  if (v == 0) {
+    const char* s = std::getenv("MOE_SWAP_KA");
+    v = (s && std::atoi(s) == 2) ? 2 : 1;
+  }
+  return v;
+}
+
+int gemm_swap_chunk() { return swap_ka() == 2 ? 32 : 64; }
+
+template <Proj P, bool FP8>
+static cudaError_t launch_swap(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a,
+                               int grid, cudaStream_t st) {
+  if (gemm_swap_chunk() == 64) return launch_one<Orient::kSwap, P, FP8, 1, 64>(tw, tx, a, grid, st);
+  if (a.katoms % 2 == 0) return launch_one<Orient::kSwap, P, FP8, 2, 32>(tw, tx, a, grid, st);
+  return launch_one<Orient::kSwap, P, FP8, 1, 32>(tw, tx, a, grid, st);
 }
 
 cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tw, const CUtensorMap& tx,
                         const GemmArgs& a, int grid, cudaStream_t st) {
   if (o == Orient::kSwap) {
     if (p == Proj::kW13)
-      return fp8 ? launch_one<Orient::kSwap, Proj::kW13, true>(tw, tx, a, grid, st)
-                 : launch_one<Orient::kSwap, Proj::kW13, false>(tw, tx, a, grid, st);
-    return fp8 ? launch_one<Orient::kSwap, Proj::kW2, true>(tw, tx, a, grid, st)
-               : launch_one<Orient::kSwap, Proj::kW2, false>(tw, tx, a, grid, st);
+      return fp8 ? launch_swap<Proj::kW13, true>(tw, tx, a, grid, st)
+                 : launch_swap<Proj::kW13, false>(tw, tx, a, grid, st);
+    return fp8 ? launch_swap<Proj::kW2, true>(tw, tx, a, grid, st)
+               : launch_swap<Proj::kW2, false>(tw, tx, a, grid, st);
   }
   if (p == Proj::kW13)
-    return fp8 ? launch_one<Orient::kNormal, Proj::kW13, true>(tw, tx, a, grid, st)
-               : launch_one<Orient::kNormal, Proj::kW13, false>(tw, tx, a, grid, st);
-  return fp8 ? launch_one<Orient::kNormal, Proj::kW2, true>(tw, tx, a, grid, st)
-             : launch_one<Orient::kNormal, Proj::kW2, false>(tw, tx, a, grid, st);
+    return fp8 ? launch_one<Orient::kNormal, Proj::kW13, true, 1, 0>(tw, tx, a, grid, st)
+               : launch_one<Orient::kNormal, Proj::kW13, false, 1, 0>(tw, tx, a, grid, st);
+  return fp8 ? launch_one<Orient::kNormal, Proj::kW2, true, 1, 0>(tw, tx, a, grid, st)
+             : launch_one<Orient::kNormal, Proj::kW2, false, 1, 0>(tw, tx, a, grid, st);
 }
 
 int gemm_token_box_rows(Orient o) { return o == Orient::kSwap ? kTokenBox : kNormalTokens; }

@@ -9,6 +9,38 @@
 
 namespace moe {
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes`, once per
+// (kernel, device); later calls with the same or a smaller size do nothing.
+cudaError_t set_smem_limit_once(const void* kernel, int bytes);
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel on the stream is still running, and must execute
+// griddepcontrol.wait (pdl_wait) before it reads anything that kernel wrote.
+template <typename... KParams, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KParams...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KParams>(args)...);
+}
+
+#ifdef __CUDACC__
+// Device side of a programmatic launch: wait for the previous kernel's
+// results, then let the next kernel on the stream be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+#endif
+
 struct RouterArgs {
   const __nv_bfloat16* hidden;
   const __nv_bfloat16* router_w;
@@ -35,8 +67,11 @@ struct AlignArgs {
   int4* chunks_swap;
   int4* chunks_normal;
   int swap_max_count;     // experts with count <= this run swap-AB
+  int swap_chunk;         // tokens per swap-AB chunk (the swap kernels' largest N)
   const float* amax_tok;  // FP8: per-token amax|x| (NULL on bf16)
   uint32_t* hdr;
+  int* gemm_flags;        // split-tile flags of the GEMM launches, zeroed here (may be NULL)
+  int n_gemm_flags;
 };
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t st);
 
@@ -68,6 +103,8 @@ struct GemmArgs {
   const uint32_t* act_scale;   // FP8: header word with s1 (w13) or s2 (w2)
   float* amax_cta;             // FP8 w13: per-CTA amax|h|
   uint32_t* hdr;
+  float* partials;             // kMaxSlots fp32 partial tiles (split units)
+  int* flags;                  // kMaxSlots flags, zero at launch
 };
 
 enum class Orient { kSwap, kNormal };
@@ -75,6 +112,7 @@ enum class Proj { kW13, kW2 };
 cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tm_w,
                         const CUtensorMap& tm_x, const GemmArgs& a, int grid, cudaStream_t st);
 int gemm_token_box_rows(Orient o);   // rows per TMA box of the token operand
+int gemm_swap_chunk();               // largest token chunk of the swap-AB kernels
 int gemm_weight_box_rows(Orient o, Proj p);
 
 }  // namespace moe

@@ -138,31 +138,48 @@ __device__ __forceinline__ int exact_cmp(const long long (&a)[kLimbs], const lon
   return 0;
 }
 
-// fp64 logit (tier 2): exact products, fp64 sequential sums per lane, butterfly.
+// fp64 logit (tier 2): exact products, four fp64 partial sums per lane (four
+// loads in flight), then the butterfly.  Every term passes through at most
+// H/32 + 8 roundings, inside the H/32 + 16 the bound assumes.
 __device__ double fp64_logit(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
                              int H) {
   const int lane = threadIdx.x & 31;
-  double acc = 0.0;
+  const int vpr = H / 8;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   const uint4* xv = reinterpret_cast<const uint4*>(x);
   const uint4* wv = reinterpret_cast<const uint4*>(w);
-  for (int c = lane; c < H / 8; c += 32) {
-    float xf[8], wf[8];
-    unpack8(xv[c], xf);
-    unpack8(wv[c], wf);
+  for (int c0 = lane; c0 < vpr; c0 += 128) {
+    uint4 xs[4], ws[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc);
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u;
+      xs[u] = c < vpr ? xv[c] : make_uint4(0, 0, 0, 0);
+      ws[u] = c < vpr ? wv[c] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float xf[8], wf[8];
+      unpack8(xs[u], xf);
+      unpack8(ws[u], wf);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        acc[u] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[u]);
+    }
   }
-  return warp_sum_d(acc);
+  return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3]));
 }
 
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Kernel 1: logits[t, e] = sum_h x[t,h] w[e,h] + b[e] in fp32, plus ||x_t||,
-// ||w_e|| for the error bound and per-token amax|x| for FP8 activation scale.
-// CTA = TT tokens x 8 experts (one expert per warp); hidden rows staged in smem.
+// Kernel 1: logits[t, e] = sum_h x[t,h] w[e,h] + b[e], accumulated in fp64
+// (F64, decode-sized calls: the error bound then shrinks to the fp32 rounding
+// of the stored logit) or fp32 (large calls), stored as fp32; plus ||x_t||,
+// ||w_e|| for the error bound and per-token amax|x| for the FP8 activation
+// scale.  CTA = TT tokens x 8 experts (one expert per warp), hidden rows
+// staged in smem, four 16-byte router-row loads in flight per lane.
 // ---------------------------------------------------------------------------
-template <int TT>
+template <int TT, bool F64>
 __global__ void __launch_bounds__(256) router_logits_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
@@ -173,9 +190,35 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
   const int nt = min(TT, T - t0);
   const int vpr = H / 8;   // 16-byte vectors per row
   const uint4* hv = reinterpret_cast<const uint4*>(hidden);
-  for (int i = threadIdx.x; i < TT * vpr; i += blockDim.x) {
-    const int r = i / vpr;
-    sx[i] = r < nt ? hv[static_cast<size_t>(t0 + r) * vpr + (i - r * vpr)] : make_uint4(0, 0, 0, 0);
+  const int e = blockIdx.y * 8 + warp;
+  const bool has_e = e < E;
+  const uint4* wrow = reinterpret_cast<const uint4*>(router_w) + static_cast<size_t>(has_e ? e : 0) * vpr;
+  constexpr int U = 8;     // 16-byte router-row loads in flight per lane
+
+  pdl_wait();
+  pdl_launch_next();
+  // the first U vectors of this warp's router row are requested before the
+  // token rows are staged, so both sets of loads are in flight together
+  uint4 wv[U];
+#pragma unroll
+  for (int u = 0; u < U; ++u) {
+    const int c = lane + 32 * u;
+    wv[u] = (has_e && c < vpr) ? wrow[c] : make_uint4(0, 0, 0, 0);
+  }
+  for (int i0 = threadIdx.x; i0 < TT * vpr; i0 += 4 * blockDim.x) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      const int r = i / vpr;
+      v[u] = (i < TT * vpr && r < nt) ? hv[static_cast<size_t>(t0 + r) * vpr + (i - r * vpr)]
+                                      : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < TT * vpr) sx[i] = v[u];
+    }
   }
   __syncthreads();
 
@@ -200,32 +243,54 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
     }
   }
 
-  const int e = blockIdx.y * 8 + warp;
-  if (e >= E) return;
-  float acc[TT];
+  if (!has_e) return;
+  using Acc = typename std::conditional<F64, double, float>::type;
+  Acc acc[TT];
 #pragma unroll
-  for (int i = 0; i < TT; ++i) acc[i] = 0.f;
+  for (int i = 0; i < TT; ++i) acc[i] = Acc(0);
   float wsq = 0.f;
-  const uint4* wrow = reinterpret_cast<const uint4*>(router_w) + static_cast<size_t>(e) * vpr;
-  for (int c = lane; c < vpr; c += 32) {
-    float wf[8];
-    unpack8(wrow[c], wf);
+  for (int c0 = lane; c0 < vpr; c0 += 32 * U) {
+    if (c0 != lane) {   // the first chunk was prefetched above
 #pragma unroll
-    for (int i = 0; i < 8; ++i) wsq = fmaf(wf[i], wf[i], wsq);
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + 32 * u;
+        wv[u] = c < vpr ? wrow[c] : make_uint4(0, 0, 0, 0);
+      }
+    }
 #pragma unroll
-    for (int tt = 0; tt < TT; ++tt) {
-      float xf[8];
-      unpack8(sx[tt * vpr + c], xf);
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + 32 * u;
+      if (c >= vpr) break;
+      float wf[8];
+      unpack8(wv[u], wf);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
+      for (int i = 0; i < 8; ++i) wsq = fmaf(wf[i], wf[i], wsq);
+#pragma unroll
+      for (int tt = 0; tt < TT; ++tt) {
+        float xf[8];
+        unpack8(sx[tt * vpr + c], xf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if constexpr (F64)
+            acc[tt] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[tt]);
+          else
+            acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
+        }
+      }
     }
   }
 #pragma unroll
-  for (int tt = 0; tt < TT; ++tt) acc[tt] = warp_sum(acc[tt]);
+  for (int tt = 0; tt < TT; ++tt) {
+    if constexpr (F64)
+      acc[tt] = warp_sum_d(acc[tt]);
+    else
+      acc[tt] = warp_sum(acc[tt]);
+  }
   wsq = warp_sum(wsq);
   if (lane == 0) {
     const float b = bias ? bias[e] : 0.f;
-    for (int tt = 0; tt < nt; ++tt) logits[static_cast<size_t>(t0 + tt) * E + e] = acc[tt] + b;
+    for (int tt = 0; tt < nt; ++tt)
+      logits[static_cast<size_t>(t0 + tt) * E + e] = static_cast<float>(acc[tt] + static_cast<Acc>(b));
     if (blockIdx.x == 0) wnorm[e] = sqrtf(wsq);
   }
 }
@@ -233,21 +298,31 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 // ---------------------------------------------------------------------------
 // Kernel 2: one warp per token.  fp32 softmax, top-(k+1) by repeated warp
 // argmax, certification against the error bound, fallback tiers 2-3.
+// kPer = experts per lane (register arrays sized by the expert count).
+// acc64: the logits were accumulated in fp64 and rounded once to fp32, so
+// the bound is the fp64 summation term plus the fp32 half-ulp of the stored
+// value; otherwise the fp32 summation bound applies.
 // ---------------------------------------------------------------------------
+template <int kPer>
 __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ logits, const float* __restrict__ xnorm,
     const float* __restrict__ wnorm, const float* __restrict__ bias,
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w, int T,
-    int H, int E, int k, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+    int H, int E, int k, int acc64, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
     unsigned char* __restrict__ cand, uint32_t* __restrict__ hdr) {
-  constexpr int kPer = kMaxExperts / 32;
+  pdl_wait();
+  pdl_launch_next();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
   const int nper = (E + 31) / 32;
   const float* row = logits + static_cast<size_t>(t) * E;
   const float xn = xnorm[t];
-  const float gamma32 = static_cast<float>(H / 32 + 16) * 5.9604645e-08f * 1.0001f;
+  // gamma_n for the summation chain (n = H/32 + 16) and the relative error of
+  // the last roundings (bias add, storage to fp32)
+  const float gamma = acc64 ? static_cast<float>((H / 32 + 16) * 1.1102230246251565e-16 * 1.0001)
+                            : static_cast<float>(H / 32 + 16) * 5.9604645e-08f * 1.0001f;
+  const float ulast = acc64 ? 5.9604645e-08f : 1.1920929e-07f;
 
   float v[kPer];
   uint32_t taken = 0;
@@ -260,7 +335,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       const float lv = row[e];
       v[i] = isnan(lv) ? -FLT_MAX : lv;   // a NaN logit ranks last
       const float b = bias ? fabsf(bias[e]) : 0.f;
-      const float r = (gamma32 * xn * wnorm[e] + 1.1920929e-07f * (fabsf(v[i]) + b)) * 1.001f;
+      const float r = (gamma * xn * wnorm[e] + ulast * (fabsf(v[i]) + b)) * 1.001f;
       rmax = fmaxf(rmax, r);
       vmax = fmaxf(vmax, v[i]);
     }
@@ -408,27 +483,38 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 }
 
 // ---------------------------------------------------------------------------
-cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
-  const int tt = a.T > 256 ? 16 : 8;
-  dim3 grid((a.T + tt - 1) / tt, (a.E + 7) / 8);
-  const size_t smem = static_cast<size_t>(tt) * a.H * 2;
-  if (tt == 16) {
-    cudaFuncSetAttribute(router_logits_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    router_logits_kernel<16><<<grid, 256, smem, st>>>(a.hidden, a.router_w, a.bias, a.T, a.H,
-                                                      a.E, a.logits, a.xnorm, a.wnorm, a.amax_tok);
-  } else {
-    cudaFuncSetAttribute(router_logits_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(smem));
-    router_logits_kernel<8><<<grid, 256, smem, st>>>(a.hidden, a.router_w, a.bias, a.T, a.H, a.E,
-                                                     a.logits, a.xnorm, a.wnorm, a.amax_tok);
-  }
-  cudaError_t err = cudaGetLastError();
+template <int TT, bool F64>
+static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
+  auto kern = router_logits_kernel<TT, F64>;
+  const int smem = TT * a.H * 2;
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return err;
-  router_topk_kernel<<<(a.T + 7) / 8, 256, 0, st>>>(a.logits, a.xnorm, a.wnorm, a.bias, a.hidden,
-                                                    a.router_w, a.T, a.H, a.E, a.k, a.topk_ids,
-                                                    a.topk_w, a.cand, a.hdr);
-  return cudaGetLastError();
+  dim3 grid((a.T + TT - 1) / TT, (a.E + 7) / 8);
+  return launch_pdl(kern, grid, dim3(256), smem, st, a.hidden, a.router_w, a.bias, a.T, a.H, a.E,
+                    a.logits, a.xnorm, a.wnorm, a.amax_tok);
+}
+
+template <int kPer>
+static cudaError_t launch_topk(const RouterArgs& a, int acc64, cudaStream_t st) {
+  return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
+                    a.xnorm, a.wnorm, a.bias, a.hidden, a.router_w, a.T, a.H, a.E, a.k, acc64,
+                    a.topk_ids, a.topk_w, a.cand, a.hdr);
+}
+
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
+  // fp64 accumulation while the logit work is small (decode batches); fp32
+  // with the wider certified bound for large batches
+  const bool acc64 = static_cast<double>(a.T) * a.E * a.H <= static_cast<double>(1 << 28);
+  const bool wide = a.T > 256 && 16 * a.H * 2 <= 200 * 1024;
+  cudaError_t err;
+  if (acc64)
+    err = wide ? launch_logits<16, true>(a, st) : launch_logits<8, true>(a, st);
+  else
+    err = wide ? launch_logits<16, false>(a, st) : launch_logits<8, false>(a, st);
+  if (err != cudaSuccess) return err;
+  if (a.E <= 64) return launch_topk<2>(a, acc64 ? 1 : 0, st);
+  if (a.E <= 256) return launch_topk<8>(a, acc64 ? 1 : 0, st);
+  return launch_topk<kMaxExperts / 32>(a, acc64 ? 1 : 0, st);
 }
 
 }  // namespace moe
