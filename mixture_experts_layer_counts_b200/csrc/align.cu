@@ -7,7 +7,7 @@
 // schedule of the grouped GEMMs (token chunks per expert, per orientation)
 // and, on the FP8 path, the per-tensor activation scale s1 = amax|x| / 448.
 //
-// One CTA of 1024 threads.  Each warp owns a contiguous slice of the flat
+// One CTA (at least E threads; more warps for large T*k).  Each warp owns a contiguous slice of the flat
 // indices; a per-warp histogram (warp-match of equal experts, leader adds the
 // group size) gives every warp its starting position per expert, so the
 // scatter is stable without atomics.
@@ -20,9 +20,10 @@ namespace moe {
 
 namespace {
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
+// Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
 __device__ int block_exclusive_scan(int v, int* tmp32, int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = blockDim.x >> 5;
   int incl = v;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -32,7 +33,7 @@ __device__ int block_exclusive_scan(int v, int* tmp32, int* total) {
   if (lane == 31) tmp32[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int w = tmp32[lane];
+    int w = lane < nw ? tmp32[lane] : 0;
     int wi = w;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
@@ -51,23 +52,25 @@ __device__ int block_exclusive_scan(int v, int* tmp32, int* total) {
 }  // namespace
 
 __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
+  // blockDim.x: a multiple of 32, >= E, <= 1024
   extern __shared__ int sh[];
-  int* hist = sh;                       // [32][E]
+  int* hist = sh;                       // [warps][E]
   __shared__ int tmp32[32];
   __shared__ int total;
   __shared__ float famax[32];
   const int E = a.E;
   const int A = a.T * a.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int NW = blockDim.x >> 5;
 
   pdl_wait();
   pdl_launch_next();
-  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) hist[i] = 0;
+  for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
   if (a.gemm_flags != nullptr)
     for (int i = threadIdx.x; i < a.n_gemm_flags; i += blockDim.x) a.gemm_flags[i] = 0;
   __syncthreads();
 
-  const int per = (A + 31) / 32;
+  const int per = (A + NW - 1) / NW;
   const int beg = min(A, warp * per), end = min(A, beg + per);
   for (int base = beg; base < end; base += 32) {
     const int f = base + lane;
@@ -86,13 +89,13 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   // counts, offsets, per-warp starting positions
   int c = 0;
   if (threadIdx.x < E)
-    for (int w = 0; w < 32; ++w) c += hist[w * E + threadIdx.x];
+    for (int w = 0; w < NW; ++w) c += hist[w * E + threadIdx.x];
   const int excl = block_exclusive_scan(threadIdx.x < E ? c : 0, tmp32, &total);
   if (threadIdx.x < E) {
     a.counts[threadIdx.x] = c;
     a.offsets[threadIdx.x] = excl;
     int run = excl;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < NW; ++w) {
       const int h = hist[w * E + threadIdx.x];
       hist[w * E + threadIdx.x] = run;
       run += h;
@@ -153,7 +156,7 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
     __syncthreads();
     if (threadIdx.x == 0) {
       float mm = 0.f;
-      for (int w = 0; w < 32; ++w) mm = fmaxf(mm, famax[w]);
+      for (int w = 0; w < NW; ++w) mm = fmaxf(mm, famax[w]);
       const float s1 = mm == 0.f ? 1.0f : __fdiv_rn(mm, 448.0f);
       a.hdr[kHdrScaleS1] = __float_as_uint(s1);
     }
@@ -161,10 +164,16 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
 }
 
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(32) * a.E * sizeof(int);
+  // one thread per expert at least; 8 warps suffice for decode-sized T*k,
+  // 32 warps shorten the per-warp slices of large batches
+  const long long A = static_cast<long long>(a.T) * a.k;
+  int threads = A >= 8192 ? 1024 : 256;
+  const int e32 = (a.E + 31) / 32 * 32;
+  if (threads < e32) threads = e32;
+  const size_t smem = static_cast<size_t>(threads / 32) * a.E * sizeof(int);
   cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(align_kernel), static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(align_kernel, dim3(1), dim3(1024), smem, st, a);
+  return launch_pdl(align_kernel, dim3(1), dim3(threads), smem, st, a);
 }
 
 }  // namespace moe

@@ -40,6 +40,19 @@ cudaError_t set_smem_limit_once(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 
+int current_sm_count() {
+  constexpr int kDevices = 64;
+  static int cache[kDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;

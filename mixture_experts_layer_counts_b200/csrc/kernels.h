@@ -13,6 +13,9 @@ namespace moe {
 // (kernel, device); later calls with the same or a smaller size do nothing.
 cudaError_t set_smem_limit_once(const void* kernel, int bytes);
 
+// Multiprocessor count of the current device (cached per device).
+int current_sm_count();
+
 // Launch with programmatic stream serialisation: the kernel may be scheduled
 // while the previous kernel on the stream is still running, and must execute
 // griddepcontrol.wait (pdl_wait) before it reads anything that kernel wrote.

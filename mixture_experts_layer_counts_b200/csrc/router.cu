@@ -348,10 +348,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     if (i < nper && lane + 32 * i < E) se += expf(v[i] - vmax);
   se = warp_sum(se);
 
-  // top-(k+1) selection, warp-wide argmax per round
+  // top-(k+1) selection, warp-wide argmax per round; slot s is kept by lane
+  // s (slot 32, the extra one when k = 32, in a warp-uniform register)
   const int nsel = min(k + 1, E);
-  int sel_idx[kMaxTopK + 1];
-  float sel_v[kMaxTopK + 1];
+  int my_idx = -1;
+  float my_v = -FLT_MAX, extra_v = -FLT_MAX;
   for (int s = 0; s < nsel; ++s) {
     float bv = -FLT_MAX;
     int bi = 0x7FFFFFFF;
@@ -372,29 +373,42 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
         bi = oi;
       }
     }
-    sel_idx[s] = bi;
-    sel_v[s] = bv;
+    if (s == lane) {
+      my_idx = bi;
+      my_v = bv;
+    }
+    if (s == 32) extra_v = bv;
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
 
+  // certified when every adjacent gap among the top k+1 exceeds twice the bound
   bool certified = true;
   if (rmax > 0.f) {
     const double margin = 2.000001 * static_cast<double>(rmax);
-    for (int s = 0; s + 1 < nsel; ++s)
-      if (!(static_cast<double>(sel_v[s]) - static_cast<double>(sel_v[s + 1]) > margin))
-        certified = false;
+    const float down = __shfl_down_sync(0xffffffffu, my_v, 1);
+    const float next_v = lane == 31 ? extra_v : down;
+    const bool bad = lane + 1 < nsel &&
+                     !(static_cast<double>(my_v) - static_cast<double>(next_v) > margin);
+    certified = !__any_sync(0xffffffffu, bad);
   }
 
-  int out[kMaxTopK];
-  if (certified) {
-    for (int j = 0; j < k; ++j) out[j] = sel_idx[j];
-  } else {
+  if (!certified) {
     if (lane == 0) atomicAdd(hdr + kHdrUncertain, 1u);
+    const float kth_v = __shfl_sync(0xffffffffu, my_v, k - 1);
+    int got = 0;
+    auto put = [&](int e) {   // slot `got` takes expert e
+      if (lane == got) {
+        my_idx = e;
+        const float lv = row[e];
+        my_v = isnan(lv) ? -FLT_MAX : lv;
+      }
+      ++got;
+    };
     // ---- tier 2: candidates re-evaluated in fp64 --------------------------
     int* c_idx = reinterpret_cast<int*>(cand + static_cast<size_t>(t) * E * 16);
     int* c_ord = c_idx + E;
     double* c_val = reinterpret_cast<double*>(c_ord + E);
-    const double thr = static_cast<double>(sel_v[k - 1]) - 2.000001 * static_cast<double>(rmax);
+    const double thr = static_cast<double>(kth_v) - 2.000001 * static_cast<double>(rmax);
     int nc = 0;
     for (int i = 0; i < nper; ++i) {
       const int e = lane + 32 * i;
@@ -432,13 +446,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     __syncwarp();
     // ---- tier 3: clusters closer than the fp64 bound, ordered exactly -----
     const double margin64 = 2.000001 * r64;
-    int got = 0, pos = 0;
+    int pos = 0;
     const uint16_t* xbits = reinterpret_cast<const uint16_t*>(xrow);
     while (got < k) {
       int end = pos;
       while (end + 1 < nc && !(c_val[c_ord[end]] - c_val[c_ord[end + 1]] > margin64)) ++end;
       if (end == pos) {
-        out[got++] = c_idx[c_ord[pos]];
+        put(c_idx[c_ord[pos]]);
         pos = end + 1;
         continue;
       }
@@ -460,7 +474,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
             best_slot = m;
           }
         }
-        out[got++] = best_e;
+        put(best_e);
         __syncwarp();
         if (lane == 0) c_idx[c_ord[best_slot]] = -1;
         __syncwarp();
@@ -470,15 +484,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   }
 
   // renormalised weights of the selected experts (fp32 softmax values)
-  float p[kMaxTopK];
-  float psum = 0.f;
-  for (int j = 0; j < k; ++j) {
-    p[j] = expf(row[out[j]] - vmax) / se;
-    psum += p[j];
-  }
-  for (int j = lane; j < k; j += 32) {
-    topk_ids[static_cast<size_t>(t) * k + j] = out[j];
-    topk_w[static_cast<size_t>(t) * k + j] = p[j] / psum;
+  const float p = lane < k ? expf(my_v - vmax) / se : 0.f;
+  const float psum = warp_sum(p);
+  if (lane < k) {
+    topk_ids[static_cast<size_t>(t) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(t) * k + lane] = p / psum;
   }
 }
 
@@ -505,12 +515,26 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   // fp64 accumulation while the logit work is small (decode batches); fp32
   // with the wider certified bound for large batches
   const bool acc64 = static_cast<double>(a.T) * a.E * a.H <= static_cast<double>(1 << 28);
-  const bool wide = a.T > 256 && 16 * a.H * 2 <= 200 * 1024;
+  // tokens per CTA: the largest of 16, 8, 4, 2 that still gives two waves of
+  // CTAs (fewer tokens per CTA means more re-reads of router rows from L2, but
+  // small decode batches need the parallelism), capped by shared memory
+  const int waves2 = 2 * current_sm_count();
+  const int eblocks = (a.E + 7) / 8;
+  int tt = 1;
+  for (int c = 16; c >= 2; c /= 2) {
+    if (c * a.H * 2 <= 200 * 1024 && ((a.T + c - 1) / c) * eblocks >= waves2) {
+      tt = c;
+      break;
+    }
+  }
   cudaError_t err;
-  if (acc64)
-    err = wide ? launch_logits<16, true>(a, st) : launch_logits<8, true>(a, st);
-  else
-    err = wide ? launch_logits<16, false>(a, st) : launch_logits<8, false>(a, st);
+  switch (tt) {
+    case 16: err = acc64 ? launch_logits<16, true>(a, st) : launch_logits<16, false>(a, st); break;
+    case 8: err = acc64 ? launch_logits<8, true>(a, st) : launch_logits<8, false>(a, st); break;
+    case 4: err = acc64 ? launch_logits<4, true>(a, st) : launch_logits<4, false>(a, st); break;
+    case 2: err = acc64 ? launch_logits<2, true>(a, st) : launch_logits<2, false>(a, st); break;
+    default: err = acc64 ? launch_logits<1, true>(a, st) : launch_logits<1, false>(a, st); break;
+  }
   if (err != cudaSuccess) return err;
   if (a.E <= 64) return launch_topk<2>(a, acc64 ? 1 : 0, st);
   if (a.E <= 256) return launch_topk<8>(a, acc64 ? 1 : 0, st);
