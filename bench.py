@@ -318,6 +318,27 @@ def run_ours(args, wl, rank, world, local):
     stage_ms = {STAGES[s]: stage_sum[s - 1] / n_stage for s in range(1, N_STAGE_EVENTS)}
     del igraph
 
+    # The dominant kernel alone: a graph whose only stage events bracket the
+    # w13 GEMM (entries 3 and 4), so the kernel is timed with one event node
+    # on each side instead of eight.
+    wev = new_events(2)
+    sel = [None] * N_STAGE_EVENTS
+    sel[3], sel[4] = wev[0], wev[1]
+    torch.cuda.synchronize()
+    wgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(wgraph):
+        layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                          stage_events=sel, **fwd)
+    w13_ms = []
+    for i in range(n_stage + 3):
+        flush.zero_()
+        wgraph.replay()
+        wev[1].synchronize()
+        if i >= 3:
+            w13_ms.append(wev[0].elapsed_time(wev[1]))
+    del wgraph
+    w13_kernel_ms = statistics.mean(w13_ms)
+
     # the same step launched directly (no graph): host launch gaps included
     n_direct = min(args.steps, 500)
     dev_ = [new_events(N_STAGE_EVENTS) for _ in range(n_direct)]
@@ -347,7 +368,7 @@ def run_ours(args, wl, rank, world, local):
     e2e_value = world * T * e2e_steps / (e2e_ms * 1e-3)
 
     peak, peak_kind = peaks()
-    w13_s = stage_ms["w13"] * 1e-3
+    w13_s = w13_kernel_ms * 1e-3
     achieved = w13_bytes / w13_s / 1e9
     line = {
         "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -370,7 +391,9 @@ def run_ours(args, wl, rank, world, local):
         "roofline": {"kernel": "grouped_gemm_kernel<swap-AB, w13>", "bound": "hbm", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": kernel_traffic(args.workload), "peak_kind": peak_kind,
-                     "algorithmic_bytes_per_launch": w13_bytes},
+                     "algorithmic_bytes_per_launch": w13_bytes, "kernel_us": 1e3 * w13_kernel_ms,
+                     "timed_by": "CUDA events recorded on the launch stream right before and after the "
+                                 "w13 GEMM, inside a graph of the layer, L2 flushed per step"},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                 "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps},
         "gpu_launches": launches_per_step(wl, T) * args.steps,

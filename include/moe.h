@@ -87,6 +87,10 @@ typedef struct {
                           boundaries: start, router, align, gather, w13, requant, w2, combine */
   int force_orient;    /* 0 = per-expert choice, 1 = swap-AB for all experts,
                           2 = normal orientation for all experts (testing) */
+  int wait_timeout_us; /* limit of each bounded device-side wait (0 = 2 s) */
+  int inject_stall;    /* failure-path test: 1 makes the first gate/up GEMM CTA leave one
+                          pipeline stage unfilled, so a bounded wait expires and the call
+                          records MOE_ERR_DEVICE_TIMEOUT (the output is then undefined) */
 } moe_debug_out_t;
 
 /* Bytes of workspace moe_forward needs for this shape (0 if the shape is

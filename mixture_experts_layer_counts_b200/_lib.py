@@ -31,7 +31,7 @@ class DebugOut(C.Structure):
         ("topk_ids", C.c_void_p), ("topk_w", C.c_void_p), ("counts", C.c_void_p),
         ("offsets", C.c_void_p), ("perm", C.c_void_p), ("inv_perm", C.c_void_p),
         ("inter", C.c_void_p), ("act_scales", C.c_void_p), ("stage_events", C.c_void_p),
-        ("force_orient", C.c_int),
+        ("force_orient", C.c_int), ("wait_timeout_us", C.c_int), ("inject_stall", C.c_int),
     ]
 
 

@@ -232,6 +232,10 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g13.act_scale = hdr + kHdrScaleS1;
   g13.hdr = hdr;
   g13.partials = at<float>(ws, L.partials);
+  g13.timeout_ns = (dbg && dbg->wait_timeout_us > 0)
+                       ? static_cast<unsigned long long>(dbg->wait_timeout_us) * 1000ull
+                       : kWaitTimeoutNs;
+  g13.inject_stall = dbg ? dbg->inject_stall : 0;
   float* amax_cta = at<float>(ws, L.amax_cta);
   if (any_swap) {
     GemmArgs g = g13;
@@ -268,6 +272,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g2.wscale = w2_scale;
   g2.act_scale = hdr + kHdrScaleS2;
   g2.amax_cta = nullptr;
+  g2.inject_stall = 0;
   if (any_swap) {
     GemmArgs g = g2;
     g.chunks = at<int4>(ws, L.chunks_swap);

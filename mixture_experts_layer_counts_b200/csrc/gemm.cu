@@ -127,14 +127,15 @@ __device__ __forceinline__ void st_release(int* p, int v) {
 }
 
 // Bounded wait for a neighbour CTA's partial-tile flag.
-__device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, uint32_t* status) {
+__device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, uint32_t* status,
+                                          unsigned long long timeout_ns) {
   if (ld_acquire(flag) != 0) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (ld_acquire(flag) != 0) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
         report_status(status, MOE_DEVICE_TIMEOUT, kSiteGridBarrier);
         *abort = 1;
         return false;
@@ -212,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per-stage bookkeeping for the abort drain
     bool ok = true;
+    bool first_stage = true;
     Segments seg{my_a0, my_a1, ksteps};
     int u, kb0, kb1;
     while (ok && seg.next(u, kb0, kb1)) {
@@ -231,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         wrow0 = e * a.w_rows_per_expert + mt * C::kBN;
       }
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty)) {
+        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty, a.timeout_ns)) {
           ok = false;
           break;
         }
@@ -239,8 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(&full[stage], bytes);
         armed |= 1u << stage;
         armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+        // failure-path test: CTA 0 arms its first stage and issues no copy,
+        // so the consumer's bounded wait runs out (nothing else ever arrives)
+        const bool skip = a.inject_stall != 0 && blockIdx.x == 0 && first_stage;
+        first_stage = false;
 #pragma unroll
-        for (int ka = 0; ka < KA; ++ka) {
+        for (int ka = 0; ka < (skip ? 0 : KA); ++ka) {
           uint8_t* sa = st + ka * C::kAtomSet;
           const int kc = (kb * KA + ka) * C::kAtomElems;
           if constexpr (C::kSwap) {
@@ -268,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < C::kStages; ++s)
         if ((armed >> s) & 1u)
           mbar_wait(&full[s], (armed_parity >> s) & 1u, reinterpret_cast<volatile int*>(&dummy),
-                    a.hdr, kSiteDrainTma);
+                    a.hdr, kSiteDrainTma, a.timeout_ns);
     }
   } else if (warp == 1 && lane == 0 && active) {
     // ---------------------------------------------------------- MMA issuer --
@@ -283,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = it & 1;
       const uint32_t accph = (it >> 1) & 1;
       ++it;
-      if (!mbar_wait(&acc_empty[buf], accph ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty)) {
+      if (!mbar_wait(&acc_empty[buf], accph ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty, a.timeout_ns)) {
         ok = false;
         break;
       }
@@ -299,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t d0 = tmem_base + buf * C::kAccCols;
       const uint32_t d1 = d0 + C::kBN;
       for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&full[stage], phase, abort_flag, a.hdr, kSiteMmaFull)) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, a.hdr, kSiteMmaFull, a.timeout_ns)) {
           ok = false;
           break;
         }
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (!ok && issued) {
       int dummy = 0;
       mma_commit(drain);
-      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), a.hdr, kSiteDrainMma);
+      mbar_wait(drain, 0, reinterpret_cast<volatile int*>(&dummy), a.hdr, kSiteDrainMma, a.timeout_ns);
     }
   } else if (warp >= 2 && active) {
     // ------------------------------------------------------------ epilogue --
@@ -348,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = it & 1;
       const uint32_t accph = (it >> 1) & 1;
       ++it;
-      if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull)) break;
+      if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull, a.timeout_ns)) break;
       tc_fence_after();
       const int4 ch = a.chunks[u / a.mtiles];
       const int mt = u % a.mtiles;
@@ -387,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long unit_end = (static_cast<long long>(u) + 1) * ksteps;
         last = atom_owner(unit_end - 1, W, G);
         bool ok = true;
-        for (int c2 = blockIdx.x + 1; c2 <= last && ok; ++c2) ok = wait_flag(a.flags + c2, abort_flag, a.hdr);
+        for (int c2 = blockIdx.x + 1; c2 <= last && ok; ++c2) ok = wait_flag(a.flags + c2, abort_flag, a.hdr, a.timeout_ns);
         if (!ok) break;
       }
       auto add_partials = [&](float (&v)[C::kNumAcc][16], int c0) {

@@ -108,6 +108,8 @@ struct GemmArgs {
   uint32_t* hdr;
   float* partials;             // kMaxSlots fp32 partial tiles (split units)
   int* flags;                  // kMaxSlots flags, zero at launch
+  unsigned long long timeout_ns;   // limit of every bounded wait in the kernel
+  int inject_stall;            // failure-path test: CTA 0 leaves one stage unfilled
 };
 
 enum class Orient { kSwap, kNormal };

@@ -59,17 +59,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Bounded: gives up
-// after kWaitTimeoutNs of wall time (or when another role of the CTA has
+// after timeout_ns of wall time (or when another role of the CTA has
 // raised *abort), records `where` in the status word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status, uint32_t where) {
+                                          uint32_t* status, uint32_t where,
+                                          unsigned long long timeout_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > timeout_ns) {
         report_status(status, MOE_DEVICE_TIMEOUT, where);
         *abort = 1;
         return false;

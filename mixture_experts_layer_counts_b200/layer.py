@@ -60,7 +60,8 @@ def make_workspace(T, H, E, I, top_k, dtype, device="cuda") -> torch.Tensor:
 
 def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w2_scale=None,
                 out=None, workspace=None, debug: dict | None = None, stream=None,
-                force_orient: int = 0, stage_events=None) -> torch.Tensor:
+                force_orient: int = 0, stage_events=None, wait_timeout_us: int = 0,
+                inject_stall: int = 0) -> torch.Tensor:
     """out[T, H] bf16 of the fused MoE layer (see include/moe.h).
 
     ``debug``: optional dict; keys filled on return (device tensors):
@@ -84,9 +85,11 @@ def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w
         workspace = make_workspace(T, H, E, I, top_k, dt, hidden.device)
     dbg_p = None
     keep = []
-    if debug is not None or force_orient or stage_events is not None:
+    if debug is not None or force_orient or stage_events is not None or wait_timeout_us or inject_stall:
         dbg = DebugOut()
         dbg.force_orient = int(force_orient)
+        dbg.wait_timeout_us = int(wait_timeout_us)
+        dbg.inject_stall = int(inject_stall)
         if debug is not None:
             A = T * top_k
             dev = hidden.device
@@ -102,7 +105,8 @@ def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w
             for k in ("topk_ids", "topk_w", "counts", "offsets", "perm", "inv_perm", "inter", "act_scales"):
                 setattr(dbg, k, debug[k].data_ptr())
         if stage_events is not None:
-            arr = (C.c_void_p * N_STAGE_EVENTS)(*[C.c_void_p(ev.cuda_event) for ev in stage_events])
+            arr = (C.c_void_p * N_STAGE_EVENTS)(
+                *[C.c_void_p(None if ev is None else ev.cuda_event) for ev in stage_events])
             keep.append(arr)
             dbg.stage_events = C.cast(arr, C.c_void_p)
         dbg_p = C.pointer(dbg)
