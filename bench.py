@@ -419,8 +419,16 @@ def main():
     ap.add_argument("--workload", default="decode", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T of the workload (smaller cases for profiler captures)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E of the workload (smaller cases for profiler captures)")
     args = ap.parse_args()
-    wl = WORKLOADS[args.workload]
+    wl = dict(WORKLOADS[args.workload])
+    if args.tokens:
+        wl["T"] = args.tokens
+    if args.experts:
+        wl["E"] = args.experts
     if args.impl == "reference":
         # the fp64 oracle takes seconds per token: small defaults, one-token samples
         args.steps = 5 if args.steps is None else args.steps

@@ -135,11 +135,11 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   const int tno = total;
   for (int i = 0; i < nsw; ++i) {
     const int n0 = i * a.swap_chunk;
-    a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(a.swap_chunk, c - n0), 0);
+    a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(a.swap_chunk, c - n0), i);
   }
   for (int i = 0; i < nno; ++i) {
     const int n0 = i * kNormalTokens;
-    a.chunks_normal[ono + i] = make_int4(threadIdx.x, excl + n0, min(kNormalTokens, c - n0), 0);
+    a.chunks_normal[ono + i] = make_int4(threadIdx.x, excl + n0, min(kNormalTokens, c - n0), i);
   }
   if (threadIdx.x == 0) {
     a.hdr[kHdrChunksSwap] = static_cast<uint32_t>(tsw);

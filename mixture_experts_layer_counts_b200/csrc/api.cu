@@ -226,6 +226,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g13.out = fp8 ? at<void>(ws, L.h32) : inter;
   g13.ld_out = I;
   g13.perm = at<int32_t>(ws, L.perm);
+  g13.counts = at<int32_t>(ws, L.counts);
   g13.topk_w = at<float>(ws, L.topk_w);
   g13.num_assign = A;
   g13.wscale = w13_scale;

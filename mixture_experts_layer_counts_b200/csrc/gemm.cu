@@ -93,11 +93,24 @@ __device__ __forceinline__ int atom_owner(long long a, long long W, int G) {
   return static_cast<int>(((a + 1) * G - 1) / W);
 }
 
-// Walks one CTA's atom range as (unit, first atom, end atom) segments.
+// Walks one CTA's work as (unit, first atom, end atom) segments: either a
+// contiguous atom range [a, a1) (balanced split), or (rr) whole units
+// u_next, u_next + step, ... < u_end dealt round-robin.
 struct Segments {
   long long a, a1;
   int katoms;
+  bool rr;
+  long long u_next, u_end;
+  int step;
   __device__ bool next(int& u, int& kb0, int& kb1) {
+    if (rr) {
+      if (u_next >= u_end) return false;
+      u = static_cast<int>(u_next);
+      kb0 = 0;
+      kb1 = katoms;
+      u_next += step;
+      return true;
+    }
     if (a >= a1) return false;
     u = static_cast<int>(a / katoms);
     kb0 = static_cast<int>(a - static_cast<long long>(u) * katoms);
@@ -107,6 +120,28 @@ struct Segments {
     return true;
   }
 };
+
+// Unit -> (token chunk, weight tile).  Swap-AB: chunk-major.  Normal
+// orientation: inside one expert, weight tile major and token chunk minor, so
+// the token chunks that share a weight tile are consecutive units; dealt
+// round-robin, they run on neighbouring CTAs at the same time and share one
+// DRAM fetch of that tile through L2.  chunk.w = index of the chunk inside its
+// expert; the expert has ceil(counts[e] / kNormalTokens) chunks.
+template <bool kGrouped>
+__device__ __forceinline__ void unit_coords(const GemmArgs& a, int u, int4& ch, int& mt) {
+  const int cs = u / a.mtiles;   // a chunk of the unit's expert
+  if constexpr (!kGrouped) {
+    ch = a.chunks[cs];
+    mt = u - cs * a.mtiles;
+  } else {
+    const int4 s = a.chunks[cs];
+    const int c0 = cs - s.w;   // the expert's first chunk
+    const int nch = (a.counts[s.x] + kNormalTokens - 1) / kNormalTokens;
+    const int local = u - c0 * a.mtiles;
+    mt = local / nch;
+    ch = a.chunks[c0 + (local - mt * nch)];
+  }
+}
 
 __device__ __forceinline__ void grid_dependency_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -199,11 +234,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       static_cast<long long>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
   const int ksteps = a.katoms / KA;   // pipeline stages per unit
   const long long W = nunits * ksteps;
+  // Swap-AB: contiguous balanced atom ranges (units may be split across CTAs).
+  // Normal orientation: whole units dealt round-robin in the grouped order.
+  constexpr bool kRR = !C::kSwap;
   int G = static_cast<int>(W / kMinAtomsPerCta);
   G = G < 1 ? 1 : (G > static_cast<int>(gridDim.x) ? static_cast<int>(gridDim.x) : G);
-  const bool active = W > 0 && static_cast<int>(blockIdx.x) < G;
-  const long long my_a0 = active ? range_begin(W, G, blockIdx.x) : 0;
-  const long long my_a1 = active ? range_begin(W, G, blockIdx.x + 1) : 0;
+  const bool active = kRR ? static_cast<long long>(blockIdx.x) < nunits
+                          : (W > 0 && static_cast<int>(blockIdx.x) < G);
+  const long long my_a0 = (active && !kRR) ? range_begin(W, G, blockIdx.x) : 0;
+  const long long my_a1 = (active && !kRR) ? range_begin(W, G, blockIdx.x + 1) : 0;
+  const Segments seg0{my_a0, my_a1, ksteps, kRR, static_cast<long long>(blockIdx.x), nunits,
+                      static_cast<int>(gridDim.x)};
 
   if (warp == 0 && lane == 0 && active) {
     // ------------------------------------------------------- TMA producer --
@@ -214,11 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t armed = 0, armed_parity = 0;   // per-stage bookkeeping for the abort drain
     bool ok = true;
     bool first_stage = true;
-    Segments seg{my_a0, my_a1, ksteps};
+    Segments seg = seg0;
     int u, kb0, kb1;
     while (ok && seg.next(u, kb0, kb1)) {
-      const int4 ch = a.chunks[u / a.mtiles];
-      const int mt = u % a.mtiles;
+      int4 ch;
+      int mt;
+      unit_coords<kRR>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       uint32_t bytes;
       int wrow0;
@@ -283,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int it = 0;
     bool ok = true;
     bool issued = false;
-    Segments seg{my_a0, my_a1, ksteps};
+    Segments seg = seg0;
     int u, kb0, kb1;
     while (ok && seg.next(u, kb0, kb1)) {
       const int buf = it & 1;
@@ -294,7 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc_fence_after();
-      const int4 ch = a.chunks[u / a.mtiles];
+      int4 ch;
+      int mt;
+      unit_coords<kRR>(a, u, ch, mt);
       int n;
       if constexpr (C::kSwap) {
         n = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
@@ -348,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = q * 32 + lane;        // accumulator row held by this thread
     float amax = 0.f;
     int it = 0;
-    Segments seg{my_a0, my_a1, ksteps};
+    Segments seg = seg0;
     int u, kb0, kb1;
     while (seg.next(u, kb0, kb1)) {
       const int buf = it & 1;
@@ -356,8 +400,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++it;
       if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull, a.timeout_ns)) break;
       tc_fence_after();
-      const int4 ch = a.chunks[u / a.mtiles];
-      const int mt = u % a.mtiles;
+      int4 ch;
+      int mt;
+      unit_coords<kRR>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
       const int ncols = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox * kTokenBox : C::kBN;

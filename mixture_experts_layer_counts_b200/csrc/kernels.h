@@ -91,8 +91,9 @@ cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16*
                            cudaStream_t st);
 
 struct GemmArgs {
-  const int4* chunks;
+  const int4* chunks;          // {expert, first row in perm order, rows, index inside expert}
   const uint32_t* nchunks;     // header word holding the chunk count
+  const int32_t* counts;       // [E] assignments per expert (normal orientation: chunks of e)
   int mtiles;                  // weight tiles per chunk
   int katoms;                  // K / 128 bytes
   int w_rows_per_expert;       // rows of one expert in the 2-D weight view
