@@ -7,10 +7,11 @@
 // schedule of the grouped GEMMs (token chunks per expert, per orientation)
 // and, on the FP8 path, the per-tensor activation scale s1 = amax|x| / 448.
 //
-// One CTA (at least E threads; more warps for large T*k).  Each warp owns a contiguous slice of the flat
-// indices; a per-warp histogram (warp-match of equal experts, leader adds the
-// group size) gives every warp its starting position per expert, so the
-// scatter is stable without atomics.
+// One CTA (at least E threads; more warps for large T*k).  Each warp owns a
+// contiguous slice of the flat indices; a per-warp histogram (lanes with equal
+// experts found by ballots on the id bits, the lowest such lane adds the group
+// size) gives every warp its starting position per expert, so the scatter is
+// stable without atomics.
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -49,6 +50,18 @@ __device__ int block_exclusive_scan(int v, int* tmp32, int* total) {
   return r;
 }
 
+// Mask of the warp's lanes holding the same key (0 <= key < 2^nbits): one
+// ballot per key bit (cheaper than a match instruction on many distinct keys).
+__device__ __forceinline__ unsigned same_key_lanes(int key, int nbits) {
+  unsigned m = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned bal = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
@@ -70,19 +83,31 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
     for (int i = threadIdx.x; i < a.n_gemm_flags; i += blockDim.x) a.gemm_flags[i] = 0;
   __syncthreads();
 
+  // each warp walks its slice in ascending flat index, kBatch loads of 32
+  // ids in flight at a time (the walk is latency-bound otherwise)
+  constexpr int kBatch = 8;
+  const int kbits = 32 - __clz(E);   // bits of the keys 0..E (E = "no expert")
   const int per = (A + NW - 1) / NW;
   const int beg = min(A, warp * per), end = min(A, beg + per);
-  for (int base = beg; base < end; base += 32) {
-    const int f = base + lane;
-    int e = f < end ? a.topk_ids[f] : -1;
-    if (e >= E || e < -1) {
-      report_status(a.hdr, MOE_DEVICE_BOUNDS, 0x100u);
-      e = -1;
+  for (int base = beg; base < end; base += 32 * kBatch) {
+    int ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int f = base + 32 * u + lane;
+      ev[u] = f < end ? a.topk_ids[f] : -1;
     }
-    const unsigned act = __ballot_sync(0xffffffffu, true);
-    const unsigned grp = __match_any_sync(act, e);
-    if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (base + 32 * u >= end) break;   // warp-uniform
+      int e = ev[u];
+      if (e >= E || e < -1) {
+        report_status(a.hdr, MOE_DEVICE_BOUNDS, 0x100u);
+        e = -1;
+      }
+      const unsigned grp = same_key_lanes(e < 0 ? E : e, kbits);
+      if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
+      __syncwarp();
+    }
   }
   __syncthreads();
 
@@ -105,20 +130,30 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   __syncthreads();
 
   // stable scatter
-  for (int base = beg; base < end; base += 32) {
-    const int f = base + lane;
-    int e = f < end ? a.topk_ids[f] : -1;
-    if (e >= E || e < -1) e = -1;
-    const unsigned grp = __match_any_sync(0xffffffffu, e);
-    const int rank = __popc(grp & ((1u << lane) - 1u));
-    if (e >= 0) {
-      const int pos = hist[warp * E + e] + rank;
-      a.perm[pos] = f;
-      a.inv_perm[f] = pos;
+  for (int base = beg; base < end; base += 32 * kBatch) {
+    int ev[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int f = base + 32 * u + lane;
+      ev[u] = f < end ? a.topk_ids[f] : -1;
     }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
-    __syncwarp();
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (base + 32 * u >= end) break;   // warp-uniform
+      const int f = base + 32 * u + lane;
+      int e = ev[u];
+      if (e >= E || e < -1) e = -1;
+      const unsigned grp = same_key_lanes(e < 0 ? E : e, kbits);
+      const int rank = __popc(grp & ((1u << lane) - 1u));
+      if (e >= 0) {
+        const int pos = hist[warp * E + e] + rank;
+        a.perm[pos] = f;
+        a.inv_perm[f] = pos;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(grp) - 1) hist[warp * E + e] += __popc(grp);
+      __syncwarp();
+    }
   }
 
   // tile schedule: swap-AB chunks of <= swap_chunk tokens for experts

@@ -32,18 +32,35 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 }
 }  // namespace
 
-__global__ void gather_kernel(const uint4* __restrict__ hidden, const int32_t* __restrict__ perm,
-                              int A, int k, int vpr, uint4* __restrict__ xperm) {
+// Work unit = (row p, block of 256 16-byte columns); a CTA takes kU units
+// per iteration so their perm and row loads are in flight together, and no
+// per-element integer division is needed.
+__global__ void __launch_bounds__(256) gather_kernel(const uint4* __restrict__ hidden,
+                                                     const int32_t* __restrict__ perm, int A, int k,
+                                                     int vpr, uint4* __restrict__ xperm) {
   pdl_wait();
   pdl_launch_next();
   const int T = A / k;
-  const size_t n = static_cast<size_t>(A) * vpr;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int p = static_cast<int>(i / vpr);
-    const int c = static_cast<int>(i - static_cast<size_t>(p) * vpr);
-    const int t = min(max(perm[p] / k, 0), T - 1);   // perm is a bijection; clamp is a guard
-    xperm[i] = hidden[static_cast<size_t>(t) * vpr + c];
+  const int nb = (vpr + 255) / 256;   // column blocks per row
+  const int units = A * nb;
+  constexpr int kU = 4;
+  for (int u0 = blockIdx.x; u0 < units; u0 += kU * gridDim.x) {
+    int t[kU], p[kU], col[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      const int unit = min(u0 + u * static_cast<int>(gridDim.x), units - 1);
+      p[u] = unit / nb;
+      col[u] = (unit - p[u] * nb) * 256 + threadIdx.x;
+      t[u] = min(max(perm[p[u]] / k, 0), T - 1);   // perm is a bijection; clamp is a guard
+    }
+    uint4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (col[u] < vpr) v[u] = hidden[static_cast<size_t>(t[u]) * vpr + col[u]];
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (u0 + u * static_cast<int>(gridDim.x) < units && col[u] < vpr)
+        xperm[static_cast<size_t>(p[u]) * vpr + col[u]] = v[u];
   }
 }
 
@@ -100,17 +117,19 @@ __global__ void requant_kernel(const float4* __restrict__ h32, const float* __re
   }
 }
 
-__global__ void combine_kernel(const float4* __restrict__ ysc, int T, int k, int h4,
-                               uint2* __restrict__ out) {
+// Work unit = (token t, block of 256 float4 columns); per thread the k slot
+// loads are issued together and summed in slot order.
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ ysc, int T, int k,
+                                                      int h4, uint2* __restrict__ out) {
   pdl_wait();
   pdl_launch_next();
-  const size_t n = static_cast<size_t>(T) * h4;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / h4);
-    const int c = static_cast<int>(i - static_cast<size_t>(t) * h4);
+  const int nb = (h4 + 255) / 256;
+  const int units = T * nb;
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int t = unit / nb;
+    const int c = (unit - t * nb) * 256 + threadIdx.x;
+    if (c >= h4) continue;
     const float4* src = ysc + static_cast<size_t>(t) * k * h4 + c;
-    // loads of up to 8 slots are issued together; the sum stays in slot order
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int j0 = 0; j0 < k; j0 += 8) {
       float4 y[8];
@@ -133,7 +152,8 @@ __global__ void combine_kernel(const float4* __restrict__ ysc, int T, int k, int
     }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
     __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    out[i] = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+    out[static_cast<size_t>(t) * h4 + c] =
+        make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
   }
 }
 
@@ -142,11 +162,13 @@ cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int 
   const int vpr = H / 8;
   const size_t n = static_cast<size_t>(A) * vpr;
   const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
+  const int units = A * ((vpr + 255) / 256);
+  const int ggrid = std::min(units, sm_count() * 8);
   if (fp8)
     return launch_pdl(gather_quant_kernel, dim3(grid), dim3(256), 0, st,
                       reinterpret_cast<const uint4*>(hidden), perm, A, k, vpr, hdr,
                       reinterpret_cast<uint2*>(xperm));
-  return launch_pdl(gather_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const uint4*>(hidden),
+  return launch_pdl(gather_kernel, dim3(ggrid), dim3(256), 0, st, reinterpret_cast<const uint4*>(hidden),
                     perm, A, k, vpr, reinterpret_cast<uint4*>(xperm));
 }
 
@@ -161,8 +183,8 @@ cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, s
 cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
                            cudaStream_t st) {
   const int h4 = H / 4;
-  const size_t n = static_cast<size_t>(T) * h4;
-  const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 8));
+  const int units = T * ((h4 + 255) / 256);
+  const int grid = std::min(units, sm_count() * 8);
   return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(ysc), T,
                     k, h4, reinterpret_cast<uint2*>(out));
 }

@@ -67,12 +67,22 @@ struct Cfg {
   static constexpr int kNumB = (!kSwap && kDual) ? 2 : 1;
   static constexpr int kAtomSet = kNumA * kATile + kNumB * kBTile;   // one K atom of every operand
   static constexpr int kStageBytes = KA * kAtomSet;
-  static constexpr int kStagesFit = (232448 - 1280) / kStageBytes;
+  // epilogue warps: 4 (one per TMEM lane quadrant); the normal orientation
+  // uses 8, two per quadrant, each taking half of the tile's columns
+  static constexpr int kEpiWarps = kSwap ? 4 : 8;
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
+  // normal orientation: per epilogue warp a 32-row x 16-column block (rows
+  // padded to 20 words) for the coalesced store transposition
+  static constexpr int kEpiCols = 16;
+  static constexpr int kEpiLd = 20;
+  static constexpr int kEpiBytes = kSwap ? 0 : kEpiWarps * 32 * kEpiLd * 4;
+  static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kNumAcc = kDual ? 2 : 1;
   static constexpr int kAccCols = kNumAcc * kBN;               // per TMEM buffer
   static constexpr int kTmemCols = 2 * kAccCols;               // 128, 256 or 512
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes;
   static constexpr int kAtomElems = FP8 ? 128 : 64;
   static constexpr int kSlotFloats = kNumAcc * kTileM * kBN;   // one CTA's partial tile
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
@@ -82,7 +92,6 @@ struct Cfg {
   static_assert(kStages >= 2, "pipeline depth");
 };
 
-constexpr int kThreads = 192;
 constexpr int kMinAtomsPerCta = 8;   // below this, fewer CTAs share the work
 
 // Contiguous atom range of CTA c out of G over W atoms, and the CTA owning atom a.
@@ -149,8 +158,9 @@ __device__ __forceinline__ void grid_dependency_wait() {
 __device__ __forceinline__ void grid_dependents_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
-__device__ __forceinline__ void epilogue_bar() {   // the 4 epilogue warps only
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+template <int kEpiThreads>
+__device__ __forceinline__ void epilogue_bar() {   // the epilogue warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(kEpiThreads) : "memory");
 }
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
@@ -180,7 +190,7 @@ __device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, 
 }
 
 template <Orient O, Proj P, bool FP8, int KA, int BNT>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, const GemmArgs a) {
   using C = Cfg<O, P, FP8, KA, BNT>;
@@ -197,7 +207,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // 4 floats: epilogue warp amax
+  float* red = reinterpret_cast<float*>(tmem_slot + 2);   // per epilogue warp amax (<= 8)
+  float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -209,11 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 32 * C::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    red[0] = red[1] = red[2] = red[3] = 0.f;
+    for (int w = 0; w < C::kEpiWarps; ++w) red[w] = 0.f;
     fence_barrier_init();
     tma_prefetch_desc(&tm_w);
     tma_prefetch_desc(&tm_x);
@@ -227,9 +238,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  grid_dependency_wait();   // the tile schedule and activations come from earlier kernels
-  grid_dependents_launch();
-
+  // The tile schedule comes from the align kernel, which has completed by
+  // the time this grid is launched: the kernel before this one (gather,
+  // requant or an earlier GEMM) starts its dependents only after its own
+  // wait for its predecessors.  So the schedule may be read, and the weight
+  // tiles (inputs of the call, written by no kernel) fetched, before the wait
+  // for the previous kernel's activations.
   const long long nunits =
       static_cast<long long>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
   const int ksteps = a.katoms / KA;   // pipeline stages per unit
@@ -246,63 +260,103 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Segments seg0{my_a0, my_a1, ksteps, kRR, static_cast<long long>(blockIdx.x), nunits,
                       static_cast<int>(gridDim.x)};
 
-  if (warp == 0 && lane == 0 && active) {
+  const bool producer = warp == 0 && lane == 0 && active;
+  if (!producer) {   // every other thread waits for the previous kernel at once
+    grid_dependency_wait();
+    grid_dependents_launch();
+  }
+
+  if (producer) {
     // ------------------------------------------------------- TMA producer --
     const uint64_t pol_w = l2_policy_evict_first();
     const uint64_t pol_x = l2_policy_evict_last();
-    int stage = 0;
-    uint32_t phase = 0;
     uint32_t armed = 0, armed_parity = 0;   // per-stage bookkeeping for the abort drain
-    bool ok = true;
-    bool first_stage = true;
-    Segments seg = seg0;
-    int u, kb0, kb1;
-    while (ok && seg.next(u, kb0, kb1)) {
+    // Copies of one pipeline stage: kb = K step of unit u; bit 0 of `parts`
+    // issues the weight tiles, bit 1 the token tiles.  Failure-path test:
+    // CTA 0 issues nothing for its first stage, so a bounded wait runs out.
+    auto issue = [&](int stage, int u, int kb, bool first, int parts) {
       int4 ch;
       int mt;
       unit_coords<kRR>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
-      uint32_t bytes;
-      int wrow0;
-      int nbox = 0;
-      if constexpr (C::kSwap) {
-        const int nvpad = (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
-        nbox = nvpad / kTokenBox;
-        bytes = KA * (C::kNumA * C::kATile + nvpad * kAtomBytes);
-        wrow0 = e * a.w_rows_per_expert + mt * kTileM;
-      } else {
-        bytes = C::kStageBytes;
-        wrow0 = e * a.w_rows_per_expert + mt * C::kBN;
-      }
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty, a.timeout_ns)) {
-          ok = false;
-          break;
-        }
-        uint8_t* st = tiles + stage * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[stage], bytes);
-        armed |= 1u << stage;
-        armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
-        // failure-path test: CTA 0 arms its first stage and issues no copy,
-        // so the consumer's bounded wait runs out (nothing else ever arrives)
-        const bool skip = a.inject_stall != 0 && blockIdx.x == 0 && first_stage;
-        first_stage = false;
+      const int wrow0 = e * a.w_rows_per_expert + mt * (C::kSwap ? kTileM : C::kBN);
+      const int nbox = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox : 0;
+      if (a.inject_stall != 0 && blockIdx.x == 0 && first) return;
+      uint8_t* st = tiles + stage * C::kStageBytes;
 #pragma unroll
-        for (int ka = 0; ka < (skip ? 0 : KA); ++ka) {
-          uint8_t* sa = st + ka * C::kAtomSet;
-          const int kc = (kb * KA + ka) * C::kAtomElems;
-          if constexpr (C::kSwap) {
+      for (int ka = 0; ka < KA; ++ka) {
+        uint8_t* sa = st + ka * C::kAtomSet;
+        const int kc = (kb * KA + ka) * C::kAtomElems;
+        if constexpr (C::kSwap) {
+          if (parts & 1) {
             tma_load_2d(sa, &tm_w, &full[stage], kc, wrow0, pol_w);
             if constexpr (C::kDual) tma_load_2d(sa + C::kATile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+          }
+          if (parts & 2) {
             uint8_t* sb = sa + C::kNumA * C::kATile;
             for (int q = 0; q < nbox; ++q)
               tma_load_2d(sb + q * kTokenBox * kAtomBytes, &tm_x, &full[stage], kc, p0 + q * kTokenBox, pol_x);
-          } else {
-            tma_load_2d(sa, &tm_x, &full[stage], kc, p0, pol_x);
+          }
+        } else {
+          if (parts & 2) tma_load_2d(sa, &tm_x, &full[stage], kc, p0, pol_x);
+          if (parts & 1) {
             tma_load_2d(sa + C::kATile, &tm_w, &full[stage], kc, wrow0, pol_w);
             if constexpr (C::kDual)
               tma_load_2d(sa + C::kATile + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
           }
+        }
+      }
+    };
+    auto stage_bytes = [&](int u) -> uint32_t {
+      if constexpr (C::kSwap) {
+        int4 ch;
+        int mt;
+        unit_coords<kRR>(a, u, ch, mt);
+        const int nvpad = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
+        return KA * (C::kNumA * C::kATile + nvpad * kAtomBytes);
+      } else {
+        return C::kStageBytes;
+      }
+    };
+
+    // (1) before the wait: arm the first kStages stages, fetch their weights
+    int pre = 0;
+    {
+      Segments seg = seg0;
+      int u, kb0, kb1;
+      while (pre < C::kStages && seg.next(u, kb0, kb1)) {
+        const uint32_t bytes = stage_bytes(u);
+        for (int kb = kb0; kb < kb1 && pre < C::kStages; ++kb, ++pre) {
+          mbar_arrive_expect_tx(&full[pre], bytes);
+          armed |= 1u << pre;
+          issue(pre, u, kb, pre == 0, 1);
+        }
+      }
+    }
+    grid_dependency_wait();
+    grid_dependents_launch();
+
+    // (2) the token tiles of those stages, then the steady-state pipeline
+    int stage = 0;
+    uint32_t phase = 0;
+    int n = 0;
+    bool ok = true;
+    Segments seg = seg0;
+    int u, kb0, kb1;
+    while (ok && seg.next(u, kb0, kb1)) {
+      const uint32_t bytes = stage_bytes(u);
+      for (int kb = kb0; kb < kb1; ++kb, ++n) {
+        if (n < pre) {
+          issue(stage, u, kb, n == 0, 2);
+        } else {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty, a.timeout_ns)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], bytes);
+          armed |= 1u << stage;
+          armed_parity = (armed_parity & ~(1u << stage)) | (phase << stage);
+          issue(stage, u, kb, false, 3);
         }
         if (++stage == C::kStages) {
           stage = 0;
@@ -343,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (C::kSwap) {
         n = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
       } else {
-        n = C::kBN;
+        n = C::kNumAcc * C::kBN;   // 256: w13 gate + up in one MMA, w2 one tile
       }
       const uint32_t idesc = idesc_f32acc(FP8 ? 0u : 1u, kTileM, static_cast<uint32_t>(n));
       const uint32_t d0 = tmem_base + buf * C::kAccCols;
@@ -366,10 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (C::kDual)
               mma_ss<FP8>(d1, sdesc_sw128(st + C::kATile + off), sdesc_sw128(sb + off), idesc, acc);
           } else {
+            // w13: the gate and up tiles are adjacent in smem, so one MMA with
+            // N = 2 * kBN covers both; its columns [0, kBN) are the gate
+            // accumulator and [kBN, 2 kBN) the up accumulator (d1 = d0 + kBN)
             mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(st + C::kATile + off), idesc, acc);
-            if constexpr (C::kDual)
-              mma_ss<FP8>(d1, sdesc_sw128(st + off), sdesc_sw128(st + C::kATile + C::kBTile + off),
-                          idesc, acc);
           }
         }
         issued = true;
@@ -407,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
       const int ncols = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox * kTokenBox : C::kBN;
 
-      if (kb0 > 0) {
+      if (!kRR && kb0 > 0) {   // (whole units only in the round-robin schedule)
         // ---- later piece of a split unit: hand the raw accumulator over ----
         float* slot = a.partials + static_cast<size_t>(blockIdx.x) * kPartialSlotFloats;
         for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -427,14 +481,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before();
         mbar_arrive(&acc_empty[buf]);
         __threadfence();
-        epilogue_bar();
+        epilogue_bar<32 * C::kEpiWarps>();
         if (row == 0) st_release(a.flags + blockIdx.x, 1);
         continue;
       }
 
       // ---- first atoms of the unit: collect the later pieces, then finish ----
       int last = blockIdx.x;
-      if (kb1 < ksteps) {
+      if (!kRR && kb1 < ksteps) {
         const long long unit_end = (static_cast<long long>(u) + 1) * ksteps;
         last = atom_owner(unit_end - 1, W, G);
         bool ok = true;
@@ -501,61 +555,102 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       } else if constexpr (C::kDual) {
-        const bool valid = row < nv;
-        const int p = p0 + row;
+        // normal w13: h for token rows p0 + rb.., intermediate columns
+        // i0 + c0..  Warp half hx takes columns [hx kBN/2, (hx+1) kBN/2) of
+        // the gate and up accumulators.  Each 16-column piece of the warp's
+        // 32 rows is staged in smem, then written as whole row segments
+        // (bf16: 32 B, fp32: 64 B) with coalesced stores.
+        float* sw = epi + (warp - 2) * 32 * C::kEpiLd;
         const int i0 = mt * C::kBN;
-        for (int c0 = 0; c0 < C::kBN; c0 += 16) {
+        const int rb = q * 32;
+        const int hx = (warp - 2) >> 2;
+        for (int c0 = hx * (C::kBN / 2); c0 < (hx + 1) * (C::kBN / 2); c0 += C::kEpiCols) {
           float v[2][16];
           tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, v[0], v[1]);
-          add_partials(v, c0);
-          if (valid) {
-            float h[16];
+          float h[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const float gg = v[0][j] * scale, uv = v[1][j] * scale;
-              h[j] = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
-            }
-            const size_t o = static_cast<size_t>(p) * a.ld_out + i0 + c0;
-            if constexpr (FP8) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + o);
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                dst[j] = make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(h[4 * j]), fabsf(h[4 * j + 1])),
-                                         fmaxf(fabsf(h[4 * j + 2]), fabsf(h[4 * j + 3]))));
-              }
-            } else {
-              uint4 pk[2];
-              uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                __nv_bfloat162 b2 = __floats2bfloat162_rn(h[2 * j], h[2 * j + 1]);
-                pw[j] = *reinterpret_cast<uint32_t*>(&b2);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + o);
-              dst[0] = pk[0];
-              dst[1] = pk[1];
-            }
+          for (int j = 0; j < 16; ++j) {
+            const float gg = v[0][j] * scale, uv = v[1][j] * scale;
+            h[j] = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
           }
-        }
-      } else {
-        int f = row < nv ? a.perm[p0 + row] : -1;
-        const bool valid = f >= 0 && f < a.num_assign;
-        float wt = 0.f;
-        if (valid) wt = a.topk_w[f] * scale;
-        const int h0 = mt * C::kBN;
-        for (int c0 = 0; c0 < C::kBN; c0 += 16) {
-          float v[1][16];
-          tmem_ld16_wait(tbase + c0, v[0]);
-          add_partials(v, c0);
-          if (valid) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) +
-                                                    static_cast<size_t>(f) * a.ld_out + h0 + c0);
+          if constexpr (FP8) {
+            if (row < nv) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(h[j]));
+            }
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              dst[j] = make_float4(v[0][4 * j] * wt, v[0][4 * j + 1] * wt, v[0][4 * j + 2] * wt,
-                                   v[0][4 * j + 3] * wt);
+              *reinterpret_cast<float4*>(sw + lane * C::kEpiLd + 4 * j) =
+                  make_float4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+            __syncwarp();
+            // 4 lanes per row (64 B), 8 rows per instruction
+#pragma unroll
+            for (int r0 = 0; r0 < 32; r0 += 8) {
+              const int r = r0 + (lane >> 2);
+              const float4 val = *reinterpret_cast<const float4*>(sw + r * C::kEpiLd + 4 * (lane & 3));
+              if (rb + r < nv)
+                *reinterpret_cast<float4*>(static_cast<float*>(a.out) +
+                                           static_cast<size_t>(p0 + rb + r) * a.ld_out + i0 + c0 +
+                                           4 * (lane & 3)) = val;
+            }
+          } else {
+            uint32_t* su = reinterpret_cast<uint32_t*>(sw);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              uint32_t w4[4];
+#pragma unroll
+              for (int m = 0; m < 4; ++m) {
+                __nv_bfloat162 b2 = __floats2bfloat162_rn(h[8 * j + 2 * m], h[8 * j + 2 * m + 1]);
+                w4[m] = *reinterpret_cast<uint32_t*>(&b2);
+              }
+              *reinterpret_cast<uint4*>(su + lane * C::kEpiLd + 4 * j) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            __syncwarp();
+            // 2 lanes per row (32 B), 16 rows per instruction
+#pragma unroll
+            for (int r0 = 0; r0 < 32; r0 += 16) {
+              const int r = r0 + (lane >> 1);
+              const uint4 val = *reinterpret_cast<const uint4*>(su + r * C::kEpiLd + 4 * (lane & 1));
+              if (rb + r < nv)
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                          static_cast<size_t>(p0 + rb + r) * a.ld_out + i0 + c0 +
+                                          8 * (lane & 1)) = val;
+            }
           }
+          __syncwarp();
+        }
+      } else {
+        // normal w2: router-weighted fp32 rows of the unit's tokens, each to
+        // its slot row f of ysc; warp half hx takes columns
+        // [hx kBN/2, (hx+1) kBN/2), staged per warp like the w13 epilogue.
+        float* sw = epi + (warp - 2) * 32 * C::kEpiLd;
+        const int f = row < nv ? a.perm[p0 + row] : -1;
+        const bool valid = f >= 0 && f < a.num_assign;
+        const float wt = valid ? a.topk_w[f] * scale : 0.f;
+        const int h0 = mt * C::kBN;
+        const int hx = (warp - 2) >> 2;
+        for (int c0 = hx * (C::kBN / 2); c0 < (hx + 1) * (C::kBN / 2); c0 += C::kEpiCols) {
+          float v[16];
+          tmem_ld16_wait(tbase + c0, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<float4*>(sw + lane * C::kEpiLd + 4 * j) =
+                make_float4(v[4 * j] * wt, v[4 * j + 1] * wt, v[4 * j + 2] * wt, v[4 * j + 3] * wt);
+          __syncwarp();
+          // 4 lanes per row (64 B), 8 rows per instruction
+#pragma unroll
+          for (int r0 = 0; r0 < 32; r0 += 8) {
+            const int r = r0 + (lane >> 2);
+            const int fr = __shfl_sync(0xffffffffu, f, r);
+            const float4 val = *reinterpret_cast<const float4*>(sw + r * C::kEpiLd + 4 * (lane & 3));
+            // streaming store (evict-first): the T*k fp32 rows are read once, by
+            // the combine pass, and should not push weight and token tiles
+            // that other CTAs still need out of L2
+            if (fr >= 0 && fr < a.num_assign)
+              __stcs(reinterpret_cast<float4*>(static_cast<float*>(a.out) + static_cast<size_t>(fr) * a.ld_out +
+                                               h0 + c0 + 4 * (lane & 3)), val);
+          }
+          __syncwarp();
         }
       }
       tc_fence_before();
@@ -573,8 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if constexpr (FP8 && C::kDual) {
     // every CTA of the grid writes its slot (0 when it had no work)
-    if (threadIdx.x == 0)
-      a.amax_cta[blockIdx.x] = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    if (threadIdx.x == 0) {
+      float m = 0.f;
+      for (int w = 0; w < C::kEpiWarps; ++w) m = fmaxf(m, red[w]);
+      a.amax_cta[blockIdx.x] = m;
+    }
   }
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
 }
@@ -586,7 +684,7 @@ static cudaError_t launch_one(const CUtensorMap& tw, const CUtensorMap& tx, cons
   auto kern = grouped_gemm_kernel<O, P, FP8, KA, BNT>;
   cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::kSmemBytes);
   if (err != cudaSuccess) return err;
-  return launch_pdl(kern, dim3(grid), dim3(kThreads), C::kSmemBytes, st, tw, tx, a);
+  return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, st, tw, tx, a);
 }
 
 // Swap-AB pipeline shape: K atoms per stage (MOE_SWAP_KA=1|2, read once).

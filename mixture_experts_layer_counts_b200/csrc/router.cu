@@ -7,8 +7,10 @@
 //   1. fp32 logits with a rigorous error bound.  Products of two bf16 values
 //      are exact in fp32, so each logit carries only summation error,
 //      |err| <= gamma_n * sum|x*w| <= gamma_n * ||x|| * ||w|| (n = the
-//      longest chain of roundings: H/32 sequential FMAs per lane plus the
-//      5-level warp butterfly), plus one rounding for the bias.
+//      longest chain of roundings of the logit kernel that ran: H/32
+//      sequential FMAs per lane plus the 5-level warp butterfly, or 64-term
+//      blocks summed in sequence for the tiled large-batch kernel), plus one
+//      rounding for the bias.
 //   2. A token whose top-(k+1) ordering is not separated by twice that bound
 //      re-evaluates only its candidate experts in fp64 (bound ~1e-16 rel).
 //   3. Candidates still within 2x the fp64 bound of each other are ordered by
@@ -296,6 +298,158 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Kernel 1b (large batches): the same logits as a register-tiled fp32 SIMT
+// GEMM.  CTA = 64 tokens x 64 experts, 256 threads, each thread 4 tokens x 4
+// experts; K in tiles of 64 staged as fp32 in smem (converted once per CTA),
+// the next tile's bf16 rows prefetched into registers while this one is
+// multiplied.  Blocked summation bounds the error: each output sums a tile's
+// 64 exact products in one FMA chain (63 roundings) and adds the tile sum to
+// its total (H/64 - 1 roundings), so every term sees at most H/64 + 62
+// roundings (the bound handed to the top-k kernel uses H/64 + 64).  The
+// norms and per-token amax|x| come from the staged values: token rows in the
+// CTAs of expert tile 0, router rows in the CTAs of token tile 0.
+// ---------------------------------------------------------------------------
+constexpr int kLgT = 64;          // tokens per CTA
+constexpr int kLgE = 64;          // experts per CTA
+constexpr int kLgK = 64;          // K per tile
+constexpr int kLgLd = kLgK + 4;   // smem row stride (floats): rows 4 banks apart
+
+__global__ void __launch_bounds__(256) router_logits_tiled_kernel(
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
+    const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
+  extern __shared__ float4 lg_smem[];
+  float* xs = reinterpret_cast<float*>(lg_smem);    // [2][kLgT][kLgLd]
+  float* wsm = xs + 2 * kLgT * kLgLd;               // [2][kLgE][kLgLd]
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * kLgT, e0 = blockIdx.y * kLgE;
+  const int vpr = H / 8;
+  const uint4* hv = reinterpret_cast<const uint4*>(hidden);
+  const uint4* rv = reinterpret_cast<const uint4*>(router_w);
+  // staging map: 512 16-byte vectors per operand tile, two per thread:
+  // row r0 (and r0 + 32), vector q of the row's 8
+  const int q = tid & 7, r0 = tid >> 3;
+  const bool xrow_ok[2] = {t0 + r0 < T, t0 + r0 + 32 < T};
+  const bool wrow_ok[2] = {e0 + r0 < E, e0 + r0 + 32 < E};
+  const bool do_xn = blockIdx.y == 0, do_wn = blockIdx.x == 0;
+  float xss[2] = {0.f, 0.f}, xam[2] = {0.f, 0.f}, wss[2] = {0.f, 0.f};
+  uint4 px[2], pw[2];
+  auto fetch = [&](int kt) {
+    const int c = kt * (kLgK / 8) + q;
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      px[s] = xrow_ok[s] ? hv[static_cast<size_t>(t0 + r0 + 32 * s) * vpr + c] : make_uint4(0, 0, 0, 0);
+      pw[s] = wrow_ok[s] ? rv[static_cast<size_t>(e0 + r0 + 32 * s) * vpr + c] : make_uint4(0, 0, 0, 0);
+    }
+  };
+  auto stage = [&](int buf) {
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      float f[8], g[8];
+      unpack8(px[s], f);
+      unpack8(pw[s], g);
+      if (do_xn) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          xss[s] = fmaf(f[i], f[i], xss[s]);
+          xam[s] = fmaxf(xam[s], fabsf(f[i]));
+        }
+      }
+      if (do_wn) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wss[s] = fmaf(g[i], g[i], wss[s]);
+      }
+      float4* dx = reinterpret_cast<float4*>(xs + (buf * kLgT + r0 + 32 * s) * kLgLd + 8 * q);
+      float4* dw = reinterpret_cast<float4*>(wsm + (buf * kLgE + r0 + 32 * s) * kLgLd + 8 * q);
+      dx[0] = make_float4(f[0], f[1], f[2], f[3]);
+      dx[1] = make_float4(f[4], f[5], f[6], f[7]);
+      dw[0] = make_float4(g[0], g[1], g[2], g[3]);
+      dw[1] = make_float4(g[4], g[5], g[6], g[7]);
+    }
+  };
+
+  pdl_wait();
+  pdl_launch_next();
+  // compute map: a warp covers 4 token rows x 8 expert rows, so each of its
+  // 16-byte smem loads touches 4 (x) or 8 (w) distinct rows in distinct banks
+  const int warp = tid >> 5, lane = tid & 31;
+  const int tx = (lane & 7) | ((warp & 1) << 3);   // experts tx + 16 j
+  const int ty = (lane >> 3) + 4 * (warp >> 1);    // tokens ty + 16 i
+  float acc[4][4], blk[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  const int nkt = H / kLgK;
+  fetch(0);
+  stage(0);
+  __syncthreads();
+  for (int kt = 0; kt < nkt; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nkt) fetch(kt + 1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) blk[i][j] = 0.f;
+    const float* xb = xs + buf * kLgT * kLgLd;
+    const float* wb = wsm + buf * kLgE * kLgLd;
+#pragma unroll 4
+    for (int kq = 0; kq < kLgK / 4; ++kq) {
+      float4 xa[4], wa[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xa[i] = *reinterpret_cast<const float4*>(xb + (ty + 16 * i) * kLgLd + 4 * kq);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wa[j] = *reinterpret_cast<const float4*>(wb + (tx + 16 * j) * kLgLd + 4 * kq);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          blk[i][j] = fmaf(xa[i].x, wa[j].x, blk[i][j]);
+          blk[i][j] = fmaf(xa[i].y, wa[j].y, blk[i][j]);
+          blk[i][j] = fmaf(xa[i].z, wa[j].z, blk[i][j]);
+          blk[i][j] = fmaf(xa[i].w, wa[j].w, blk[i][j]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += blk[i][j];
+    if (kt + 1 < nkt) stage(buf ^ 1);
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int e = e0 + tx + 16 * j;
+    if (e >= E) continue;
+    const float b = bias ? bias[e] : 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + ty + 16 * i;
+      if (t < T) logits[static_cast<size_t>(t) * E + e] = acc[i][j] + b;
+    }
+  }
+  // norms: the 8 threads of a staging row are 8 consecutive lanes
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+#pragma unroll
+    for (int m = 1; m < 8; m <<= 1) {
+      xss[s] += __shfl_xor_sync(0xffffffffu, xss[s], m);
+      xam[s] = fmaxf(xam[s], __shfl_xor_sync(0xffffffffu, xam[s], m));
+      wss[s] += __shfl_xor_sync(0xffffffffu, wss[s], m);
+    }
+    if (q == 0) {
+      if (do_xn && xrow_ok[s]) {
+        xnorm[t0 + r0 + 32 * s] = sqrtf(xss[s]);
+        amax_tok[t0 + r0 + 32 * s] = xam[s];
+      }
+      if (do_wn && wrow_ok[s]) wnorm[e0 + r0 + 32 * s] = sqrtf(wss[s]);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Kernel 2: one warp per token.  fp32 softmax, top-(k+1) by repeated warp
 // argmax, certification against the error bound, fallback tiers 2-3.
 // kPer = experts per lane (register arrays sized by the expert count).
@@ -308,7 +462,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ logits, const float* __restrict__ xnorm,
     const float* __restrict__ wnorm, const float* __restrict__ bias,
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w, int T,
-    int H, int E, int k, int acc64, int32_t* __restrict__ topk_ids, float* __restrict__ topk_w,
+    int H, int E, int k, int acc64, int nchain, int32_t* __restrict__ topk_ids,
+    float* __restrict__ topk_w,
     unsigned char* __restrict__ cand, uint32_t* __restrict__ hdr) {
   pdl_wait();
   pdl_launch_next();
@@ -318,11 +473,13 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   const int nper = (E + 31) / 32;
   const float* row = logits + static_cast<size_t>(t) * E;
   const float xn = xnorm[t];
-  // gamma_n for the summation chain (n = H/32 + 16) and the relative error of
-  // the last roundings (bias add, storage to fp32)
-  const float gamma = acc64 ? static_cast<float>((H / 32 + 16) * 1.1102230246251565e-16 * 1.0001)
-                            : static_cast<float>(H / 32 + 16) * 5.9604645e-08f * 1.0001f;
+  // gamma_n for the summation chain (n = nchain, the logit kernel's longest
+  // chain of roundings), the relative error of the last roundings (bias add,
+  // storage to fp32), and H products that might underflow (2^-149 each)
+  const float gamma = acc64 ? static_cast<float>(nchain * 1.1102230246251565e-16 * 1.0001)
+                            : static_cast<float>(nchain) * 5.9604645e-08f * 1.0001f;
   const float ulast = acc64 ? 5.9604645e-08f : 1.1920929e-07f;
+  const float tiny = static_cast<float>(H) * 1.4012985e-45f;
 
   float v[kPer];
   uint32_t taken = 0;
@@ -335,7 +492,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       const float lv = row[e];
       v[i] = isnan(lv) ? -FLT_MAX : lv;   // a NaN logit ranks last
       const float b = bias ? fabsf(bias[e]) : 0.f;
-      const float r = (gamma * xn * wnorm[e] + ulast * (fabsf(v[i]) + b)) * 1.001f;
+      const float r = (gamma * xn * wnorm[e] + ulast * (fabsf(v[i]) + b) + tiny) * 1.001f;
       rmax = fmaxf(rmax, r);
       vmax = fmaxf(vmax, v[i]);
     }
@@ -505,40 +662,60 @@ static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
 }
 
 template <int kPer>
-static cudaError_t launch_topk(const RouterArgs& a, int acc64, cudaStream_t st) {
+static cudaError_t launch_topk(const RouterArgs& a, int acc64, int nchain, cudaStream_t st) {
   return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
                     a.xnorm, a.wnorm, a.bias, a.hidden, a.router_w, a.T, a.H, a.E, a.k, acc64,
-                    a.topk_ids, a.topk_w, a.cand, a.hdr);
+                    nchain, a.topk_ids, a.topk_w, a.cand, a.hdr);
+}
+
+static cudaError_t launch_logits_tiled(const RouterArgs& a, cudaStream_t st) {
+  auto kern = router_logits_tiled_kernel;
+  const int smem = 2 * (kLgT + kLgE) * kLgLd * 4;
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((a.T + kLgT - 1) / kLgT, (a.E + kLgE - 1) / kLgE);
+  return launch_pdl(kern, grid, dim3(256), smem, st, a.hidden, a.router_w, a.bias, a.T, a.H, a.E,
+                    a.logits, a.xnorm, a.wnorm, a.amax_tok);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   // fp64 accumulation while the logit work is small (decode batches); fp32
   // with the wider certified bound for large batches
   const bool acc64 = static_cast<double>(a.T) * a.E * a.H <= static_cast<double>(1 << 28);
-  // tokens per CTA: the largest of 16, 8, 4, 2 that still gives two waves of
-  // CTAs (fewer tokens per CTA means more re-reads of router rows from L2, but
-  // small decode batches need the parallelism), capped by shared memory
-  const int waves2 = 2 * current_sm_count();
-  const int eblocks = (a.E + 7) / 8;
-  int tt = 1;
-  for (int c = 16; c >= 2; c /= 2) {
-    if (c * a.H * 2 <= 200 * 1024 && ((a.T + c - 1) / c) * eblocks >= waves2) {
-      tt = c;
-      break;
-    }
-  }
   cudaError_t err;
-  switch (tt) {
-    case 16: err = acc64 ? launch_logits<16, true>(a, st) : launch_logits<16, false>(a, st); break;
-    case 8: err = acc64 ? launch_logits<8, true>(a, st) : launch_logits<8, false>(a, st); break;
-    case 4: err = acc64 ? launch_logits<4, true>(a, st) : launch_logits<4, false>(a, st); break;
-    case 2: err = acc64 ? launch_logits<2, true>(a, st) : launch_logits<2, false>(a, st); break;
-    default: err = acc64 ? launch_logits<1, true>(a, st) : launch_logits<1, false>(a, st); break;
+  int nchain;
+  if (!acc64 && a.E >= 32) {
+    // large batch: register-tiled fp32 GEMM (blocked summation, see above)
+    err = launch_logits_tiled(a, st);
+    nchain = a.H / kLgK + 64;
+  } else {
+    // tokens per CTA: the largest of 16, 8, 4, 2 that still gives two waves
+    // of CTAs (fewer tokens per CTA means more re-reads of router rows from
+    // L2, but small decode batches need the parallelism), capped by shared
+    // memory.  Chain: H/32 FMAs per lane plus the 5-level butterfly.
+    const int waves2 = 2 * current_sm_count();
+    const int eblocks = (a.E + 7) / 8;
+    int tt = 1;
+    for (int c = 16; c >= 2; c /= 2) {
+      if (c * a.H * 2 <= 200 * 1024 && ((a.T + c - 1) / c) * eblocks >= waves2) {
+        tt = c;
+        break;
+      }
+    }
+    switch (tt) {
+      case 16: err = acc64 ? launch_logits<16, true>(a, st) : launch_logits<16, false>(a, st); break;
+      case 8: err = acc64 ? launch_logits<8, true>(a, st) : launch_logits<8, false>(a, st); break;
+      case 4: err = acc64 ? launch_logits<4, true>(a, st) : launch_logits<4, false>(a, st); break;
+      case 2: err = acc64 ? launch_logits<2, true>(a, st) : launch_logits<2, false>(a, st); break;
+      default: err = acc64 ? launch_logits<1, true>(a, st) : launch_logits<1, false>(a, st); break;
+    }
+    nchain = a.H / 32 + 16;
   }
   if (err != cudaSuccess) return err;
-  if (a.E <= 64) return launch_topk<2>(a, acc64 ? 1 : 0, st);
-  if (a.E <= 256) return launch_topk<8>(a, acc64 ? 1 : 0, st);
-  return launch_topk<kMaxExperts / 32>(a, acc64 ? 1 : 0, st);
+  const int f64 = acc64 ? 1 : 0;
+  if (a.E <= 64) return launch_topk<2>(a, f64, nchain, st);
+  if (a.E <= 256) return launch_topk<8>(a, f64, nchain, st);
+  return launch_topk<kMaxExperts / 32>(a, f64, nchain, st);
 }
 
 }  // namespace moe

@@ -58,6 +58,27 @@ def _route_pair(x, wr, k, bias=None):
     return ids.cpu().numpy(), w.cpu().numpy(), rids, rw, n_exact
 
 
+@pytest.mark.parametrize("T,H,E,k,bias,dup", [
+    (1000, 4096, 96, 8, True, False),     # ragged token and expert tiles, H/64 = 64 K tiles
+    (20000, 128, 128, 4, False, False),   # two K tiles, many token tiles
+    (600, 8192, 64, 6, False, True),      # exact ties between duplicated router rows
+])
+def test_route_large_batch_tiled(cuda_ok, T, H, E, k, bias, dup):
+    # T * E * H > 2^28 with E >= 32: logits from the register-tiled fp32 kernel
+    assert T * E * H > 2 ** 28 and E >= 32
+    rng = np.random.default_rng(T + H + E)
+    x = rng.standard_normal((T, H))
+    wr = rng.standard_normal((E, H)) * 0.05
+    if dup:
+        wr[5] = wr[2]
+        wr[40] = wr[17]
+        wr[41] = wr[17]
+    b = (rng.standard_normal(E) * 0.5).astype(np.float32) if bias else None
+    ids, w, rids, rw, _ = _route_pair(x, wr, k, b)
+    assert np.array_equal(ids, rids)
+    assert np.abs(w - rw).max() <= WEIGHT_ATOL
+
+
 def test_route_duplicate_rows_lower_index_first(cuda_ok):
     rng = np.random.default_rng(0)
     H, E, k = 256, 40, 6
