@@ -64,7 +64,13 @@ __device__ __forceinline__ unsigned same_key_lanes(int key, int nbits) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
+// mode 0: the whole job in one CTA.  Large T*k runs as two grids over
+// slices of the flat index range, one slice per CTA: mode 1 writes each
+// CTA's per-expert counts to a.slice_hist; mode 2 recomputes its own slice's
+// per-warp counts, places the slice after the earlier slices' assignments of
+// each expert (prefix over slice_hist) and scatters; its CTA 0 also writes
+// counts, offsets, the tile schedule and the FP8 scale.
+__global__ void __launch_bounds__(1024) align_kernel(AlignArgs a, int mode, int slice) {
   // blockDim.x: a multiple of 32, >= E, <= 1024
   extern __shared__ int sh[];
   int* hist = sh;                       // [warps][E]
@@ -75,20 +81,23 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   const int A = a.T * a.k;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int NW = blockDim.x >> 5;
+  const int cbeg = mode == 0 ? 0 : min(A, static_cast<int>(blockIdx.x) * slice);
+  const int cend = mode == 0 ? A : min(A, cbeg + slice);
+  const bool lead = mode == 0 || (mode == 2 && blockIdx.x == 0);   // writes the shared outputs
 
   pdl_wait();
   pdl_launch_next();
   for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
-  if (a.gemm_flags != nullptr)
+  if (a.gemm_flags != nullptr && mode != 2 && blockIdx.x == 0)
     for (int i = threadIdx.x; i < a.n_gemm_flags; i += blockDim.x) a.gemm_flags[i] = 0;
   __syncthreads();
 
-  // each warp walks its slice in ascending flat index, kBatch loads of 32
-  // ids in flight at a time (the walk is latency-bound otherwise)
+  // each warp walks its part of the slice in ascending flat index, kBatch
+  // loads of 32 ids in flight at a time
   constexpr int kBatch = 8;
   const int kbits = 32 - __clz(E);   // bits of the keys 0..E (E = "no expert")
-  const int per = (A + NW - 1) / NW;
-  const int beg = min(A, warp * per), end = min(A, beg + per);
+  const int per = (cend - cbeg + NW - 1) / NW;
+  const int beg = min(cend, cbeg + warp * per), end = min(cend, beg + per);
   for (int base = beg; base < end; base += 32 * kBatch) {
     int ev[kBatch];
 #pragma unroll
@@ -101,7 +110,7 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
       if (base + 32 * u >= end) break;   // warp-uniform
       int e = ev[u];
       if (e >= E || e < -1) {
-        report_status(a.hdr, MOE_DEVICE_BOUNDS, 0x100u);
+        if (mode != 2) report_status(a.hdr, MOE_DEVICE_BOUNDS, 0x100u);
         e = -1;
       }
       const unsigned grp = same_key_lanes(e < 0 ? E : e, kbits);
@@ -111,22 +120,42 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
   }
   __syncthreads();
 
+  if (mode == 1) {   // slice totals per expert
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int c = 0;
+      for (int w = 0; w < NW; ++w) c += hist[w * E + e];
+      a.slice_hist[static_cast<size_t>(blockIdx.x) * E + e] = c;
+    }
+    return;
+  }
+
   // counts, offsets, per-warp starting positions
-  int c = 0;
-  if (threadIdx.x < E)
-    for (int w = 0; w < NW; ++w) c += hist[w * E + threadIdx.x];
+  int c = 0, before = 0;   // count of expert threadIdx.x; its assignments in earlier slices
+  if (threadIdx.x < E) {
+    if (mode == 0) {
+      for (int w = 0; w < NW; ++w) c += hist[w * E + threadIdx.x];
+    } else {
+      for (int b = 0; b < static_cast<int>(gridDim.x); ++b) {
+        const int h = a.slice_hist[static_cast<size_t>(b) * E + threadIdx.x];
+        if (b < static_cast<int>(blockIdx.x)) before += h;
+        c += h;
+      }
+    }
+  }
   const int excl = block_exclusive_scan(threadIdx.x < E ? c : 0, tmp32, &total);
   if (threadIdx.x < E) {
-    a.counts[threadIdx.x] = c;
-    a.offsets[threadIdx.x] = excl;
-    int run = excl;
+    if (lead) {
+      a.counts[threadIdx.x] = c;
+      a.offsets[threadIdx.x] = excl;
+    }
+    int run = excl + before;
     for (int w = 0; w < NW; ++w) {
       const int h = hist[w * E + threadIdx.x];
       hist[w * E + threadIdx.x] = run;
       run += h;
     }
   }
-  if (threadIdx.x == 0) a.offsets[E] = total;
+  if (threadIdx.x == 0 && lead) a.offsets[E] = total;
   __syncthreads();
 
   // stable scatter
@@ -155,6 +184,7 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
       __syncwarp();
     }
   }
+  if (!lead) return;
 
   // tile schedule: swap-AB chunks of <= swap_chunk tokens for experts
   // with count <= swap_max_count, normal-orientation tiles of kNormalTokens
@@ -199,16 +229,31 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a) {
 }
 
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t st) {
-  // one thread per expert at least; 8 warps suffice for decode-sized T*k,
-  // 32 warps shorten the per-warp slices of large batches
   const long long A = static_cast<long long>(a.T) * a.k;
-  int threads = A >= 8192 ? 1024 : 256;
   const int e32 = (a.E + 31) / 32 * 32;
+  auto kern = align_kernel;
+  if (A < kAlignSliceMin || a.slice_hist == nullptr) {
+    // one CTA: 8 warps suffice for decode-sized T*k, 32 shorten the
+    // per-warp walks of mid-sized batches
+    int threads = A >= 8192 ? 1024 : 256;
+    if (threads < e32) threads = e32;
+    const size_t smem = static_cast<size_t>(threads / 32) * a.E * sizeof(int);
+    cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+    return launch_pdl(kern, dim3(1), dim3(threads), smem, st, a, 0, 0);
+  }
+  // two grids over slices of >= kAlignSliceMin / 8 assignments, at most kAlignMaxSlices
+  long long nb = (A + kAlignSliceMin / 8 - 1) / (kAlignSliceMin / 8);
+  if (nb > kAlignMaxSlices) nb = kAlignMaxSlices;
+  const int slice = static_cast<int>((A + nb - 1) / nb);
+  int threads = 256;
   if (threads < e32) threads = e32;
   const size_t smem = static_cast<size_t>(threads / 32) * a.E * sizeof(int);
-  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(align_kernel), static_cast<int>(smem));
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  return launch_pdl(align_kernel, dim3(1), dim3(threads), smem, st, a);
+  err = launch_pdl(kern, dim3(static_cast<int>(nb)), dim3(threads), smem, st, a, 1, slice);
+  if (err != cudaSuccess) return err;
+  return launch_pdl(kern, dim3(static_cast<int>(nb)), dim3(threads), smem, st, a, 2, slice);
 }
 
 }  // namespace moe

@@ -201,7 +201,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 router_bias, T, H, E, k,
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
-                at<unsigned char>(ws, L.cand), hdr};
+                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit)};
   MOE_TRY(cuda_status(launch_router(ra, st)));
   record(dbg, 1, st);
 
@@ -209,7 +209,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
-               at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots};
+               at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots, at<int>(ws, L.slice_hist)};
   MOE_TRY(cuda_status(launch_align(aa, st)));
   record(dbg, 2, st);
 
@@ -366,12 +366,13 @@ moe_status_t moe_route(const void* hidden, const void* router_w, const float* ro
   if (!hidden || !router_w || !topk_ids || !topk_w || !workspace) return MOE_ERR_INVALID_ARG;
   if (!aligned16(hidden) || !aligned16(router_w) || !aligned16(workspace)) return MOE_ERR_MISALIGNED;
   const Layout L = make_layout(T, H, E, 128, top_k, false);
-  if (workspace_bytes < L.cand + static_cast<size_t>(T) * E * 16) return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < L.rsplit + router_split_floats(T, E) * 4) return MOE_ERR_WORKSPACE_TOO_SMALL;
   RouterArgs ra{static_cast<const __nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(router_w),
                 router_bias, T, H, E, top_k,
                 at<float>(workspace, L.logits), at<float>(workspace, L.xnorm),
                 at<float>(workspace, L.wnorm), at<float>(workspace, L.amax_tok), topk_ids, topk_w,
-                at<unsigned char>(workspace, L.cand), at<uint32_t>(workspace, L.header)};
+                at<unsigned char>(workspace, L.cand), at<uint32_t>(workspace, L.header),
+                at<float>(workspace, L.rsplit)};
   return cuda_status(launch_router(ra, static_cast<cudaStream_t>(stream)));
 }
 
@@ -388,7 +389,8 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t
   AlignArgs aa{topk_ids, T, E, top_k, counts, offsets, perm, inv_perm,
                at<int4>(workspace, L.chunks_swap), at<int4>(workspace, L.chunks_normal),
                swap_threshold(), gemm_swap_chunk(), nullptr, at<uint32_t>(workspace, L.header),
-               at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots};
+               at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots,
+               at<int>(workspace, L.slice_hist)};
   return cuda_status(launch_align(aa, static_cast<cudaStream_t>(stream)));
 }
 

@@ -58,13 +58,25 @@ __device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, u
 
 // Byte offsets of every region of the caller-provided workspace.
 struct Layout {
-  size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand;
+  size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand, rsplit;
+  size_t slice_hist;
   size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, gemm_flags, partials;
   size_t xperm, inter, h32, ysc, staging_in, staging_out, total;
   int max_chunks_swap, max_chunks_normal;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Split-K router partials: up to kRouterSplits partial logit matrices and
+// partial sums for the norms and amax (see the tiled logits kernel).
+constexpr int kRouterSplits = 4;
+// moe_align: T*k at or above kAlignSliceMin runs as two grids over at most
+// kAlignMaxSlices slices (per-slice expert counts in the workspace).
+constexpr int kAlignSliceMin = 8192;
+constexpr int kAlignMaxSlices = 256;
+inline size_t router_split_floats(int T, int E) {
+  return static_cast<size_t>(kRouterSplits) * (static_cast<size_t>(T) * E + 2 * static_cast<size_t>(T) + E);
+}
 
 inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   Layout L{};
@@ -84,10 +96,12 @@ inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   L.amax_tok = take(static_cast<size_t>(T) * 4);
   L.amax_cta = take(static_cast<size_t>(kMaxGrid) * 4);
   L.cand = take(static_cast<size_t>(T) * E * 16);    // router fallback scratch
+  L.rsplit = take(router_split_floats(T, E) * 4);     // split-K router partials
   L.counts = take(static_cast<size_t>(E) * 4);
   L.offsets = take(static_cast<size_t>(E + 1) * 4);
   L.perm = take(A * 4);
   L.inv_perm = take(A * 4);
+  L.slice_hist = take(static_cast<size_t>(kAlignMaxSlices) * E * 4);
   L.max_chunks_swap = static_cast<int>(E + A / 16 + 1);   // swap chunks hold >= 16 tokens
   L.max_chunks_normal = static_cast<int>(E + A / kNormalTokens + 1);
   L.chunks_swap = take(static_cast<size_t>(L.max_chunks_swap) * 16);

@@ -57,6 +57,7 @@ struct RouterArgs {
   float* topk_w;
   unsigned char* cand;
   uint32_t* hdr;
+  float* rsplit;          // router_split_floats(T, E) floats, or NULL (no split-K)
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 
@@ -75,6 +76,7 @@ struct AlignArgs {
   uint32_t* hdr;
   int* gemm_flags;        // split-tile flags of the GEMM launches, zeroed here (may be NULL)
   int n_gemm_flags;
+  int* slice_hist;        // kAlignMaxSlices * E ints for large T*k (NULL: one CTA)
 };
 cudaError_t launch_align(const AlignArgs& a, cudaStream_t st);
 

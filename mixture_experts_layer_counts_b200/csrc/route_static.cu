@@ -101,6 +101,6 @@ extern "C" moe_status_t moe_route_static(const void* hidden, const void* router_
                 reinterpret_cast<float*>(b + L.logits), reinterpret_cast<float*>(b + L.xnorm),
                 reinterpret_cast<float*>(b + L.wnorm), reinterpret_cast<float*>(b + L.amax_tok),
                 topk_ids, topk_w, reinterpret_cast<unsigned char*>(b + L.cand),
-                reinterpret_cast<uint32_t*>(b + L.header)};
+                reinterpret_cast<uint32_t*>(b + L.header), nullptr};
   return launch_router(ra, st) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

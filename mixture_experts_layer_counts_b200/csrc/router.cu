@@ -308,6 +308,11 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
 // roundings (the bound handed to the top-k kernel uses H/64 + 64).  The
 // norms and per-token amax|x| come from the staged values: token rows in the
 // CTAs of expert tile 0, router rows in the CTAs of token tile 0.
+// Split-K (gridDim.z = S > 1, for batches whose tiles alone would leave SMs
+// idle): CTA z covers K tiles [z n/S, (z+1) n/S) and writes its partial
+// logits (no bias), partial sums of squares and partial amax to rsplit; the
+// top-k kernel adds the S partials in z order, then the bias.  Each term then
+// sees at most H/(64S) + S + 61 <= H/64 + 64 roundings.
 // ---------------------------------------------------------------------------
 constexpr int kLgT = 64;          // tokens per CTA
 constexpr int kLgE = 64;          // experts per CTA
@@ -317,7 +322,8 @@ constexpr int kLgLd = kLgK + 4;   // smem row stride (floats): rows 4 banks apar
 __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
-    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok,
+    float* __restrict__ rsplit) {
   extern __shared__ float4 lg_smem[];
   float* xs = reinterpret_cast<float*>(lg_smem);    // [2][kLgT][kLgLd]
   float* wsm = xs + 2 * kLgT * kLgLd;               // [2][kLgE][kLgLd]
@@ -381,13 +387,15 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-  const int nkt = H / kLgK;
-  fetch(0);
+  const int S = gridDim.z, z = blockIdx.z;
+  const int nkt_all = H / kLgK;
+  const int kt0 = z * nkt_all / S, nkt = (z + 1) * nkt_all / S - kt0;
+  fetch(kt0);
   stage(0);
   __syncthreads();
   for (int kt = 0; kt < nkt; ++kt) {
     const int buf = kt & 1;
-    if (kt + 1 < nkt) fetch(kt + 1);
+    if (kt + 1 < nkt) fetch(kt0 + kt + 1);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -419,6 +427,11 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
     __syncthreads();
   }
 
+  // split-K partial regions: logits [S][T][E], sum x^2 [S][T], amax [S][T], sum w^2 [S][E]
+  float* p_log = rsplit;
+  float* p_xss = rsplit + static_cast<size_t>(S) * T * E;
+  float* p_xam = p_xss + static_cast<size_t>(S) * T;
+  float* p_wss = p_xam + static_cast<size_t>(S) * T;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int e = e0 + tx + 16 * j;
@@ -427,7 +440,11 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = t0 + ty + 16 * i;
-      if (t < T) logits[static_cast<size_t>(t) * E + e] = acc[i][j] + b;
+      if (t >= T) continue;
+      if (S == 1)
+        logits[static_cast<size_t>(t) * E + e] = acc[i][j] + b;
+      else
+        p_log[(static_cast<size_t>(z) * T + t) * E + e] = acc[i][j];
     }
   }
   // norms: the 8 threads of a staging row are 8 consecutive lanes
@@ -440,11 +457,22 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
       wss[s] += __shfl_xor_sync(0xffffffffu, wss[s], m);
     }
     if (q == 0) {
+      const int t = t0 + r0 + 32 * s, e = e0 + r0 + 32 * s;
       if (do_xn && xrow_ok[s]) {
-        xnorm[t0 + r0 + 32 * s] = sqrtf(xss[s]);
-        amax_tok[t0 + r0 + 32 * s] = xam[s];
+        if (S == 1) {
+          xnorm[t] = sqrtf(xss[s]);
+          amax_tok[t] = xam[s];
+        } else {
+          p_xss[static_cast<size_t>(z) * T + t] = xss[s];
+          p_xam[static_cast<size_t>(z) * T + t] = xam[s];
+        }
       }
-      if (do_wn && wrow_ok[s]) wnorm[e0 + r0 + 32 * s] = sqrtf(wss[s]);
+      if (do_wn && wrow_ok[s]) {
+        if (S == 1)
+          wnorm[e] = sqrtf(wss[s]);
+        else
+          p_wss[static_cast<size_t>(z) * E + e] = wss[s];
+      }
     }
   }
 }
@@ -456,23 +484,56 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
 // acc64: the logits were accumulated in fp64 and rounded once to fp32, so
 // the bound is the fp64 summation term plus the fp32 half-ulp of the stored
 // value; otherwise the fp32 summation bound applies.
+// nsplit > 1: the logits kernel ran split-K; this kernel first adds the
+// token's nsplit partial logits in split order, then the bias, stores the
+// row to `logits`, and forms ||x_t||, amax|x_t| and ||w_e|| from the partial
+// sums.
 // ---------------------------------------------------------------------------
 template <int kPer>
 __global__ void __launch_bounds__(256) router_topk_kernel(
-    const float* __restrict__ logits, const float* __restrict__ xnorm,
-    const float* __restrict__ wnorm, const float* __restrict__ bias,
-    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w, int T,
-    int H, int E, int k, int acc64, int nchain, int32_t* __restrict__ topk_ids,
-    float* __restrict__ topk_w,
-    unsigned char* __restrict__ cand, uint32_t* __restrict__ hdr) {
+    float* __restrict__ logits, float* __restrict__ xnorm, const float* __restrict__ wnorm,
+    float* __restrict__ amax_tok, const float* __restrict__ rsplit, int nsplit,
+    const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
+    const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, int acc64, int nchain,
+    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
+    uint32_t* __restrict__ hdr) {
   pdl_wait();
   pdl_launch_next();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
   const int nper = (E + 31) / 32;
-  const float* row = logits + static_cast<size_t>(t) * E;
-  const float xn = xnorm[t];
+  float* row = logits + static_cast<size_t>(t) * E;
+  const float* p_xss = rsplit + static_cast<size_t>(nsplit) * T * E;
+  const float* p_xam = p_xss + static_cast<size_t>(nsplit) * T;
+  const float* p_wss = p_xam + static_cast<size_t>(nsplit) * T;
+  float xn;
+  if (nsplit > 1) {
+    float ss = 0.f, am = 0.f;
+    for (int z = 0; z < nsplit; ++z) {
+      ss += p_xss[static_cast<size_t>(z) * T + t];
+      am = fmaxf(am, p_xam[static_cast<size_t>(z) * T + t]);
+    }
+    xn = sqrtf(ss);
+    if (lane == 0) {
+      xnorm[t] = xn;
+      amax_tok[t] = am;
+    }
+    for (int e = lane; e < E; e += 32) {
+      float v = rsplit[static_cast<size_t>(t) * E + e];
+      for (int z = 1; z < nsplit; ++z) v += rsplit[(static_cast<size_t>(z) * T + t) * E + e];
+      row[e] = v + (bias ? bias[e] : 0.f);
+    }
+    __syncwarp();
+  } else {
+    xn = xnorm[t];
+  }
+  auto wnorm_of = [&](int e) -> float {
+    if (nsplit <= 1) return wnorm[e];
+    float ss = 0.f;
+    for (int z = 0; z < nsplit; ++z) ss += p_wss[static_cast<size_t>(z) * E + e];
+    return sqrtf(ss);
+  };
   // gamma_n for the summation chain (n = nchain, the logit kernel's longest
   // chain of roundings), the relative error of the last roundings (bias add,
   // storage to fp32), and H products that might underflow (2^-149 each)
@@ -492,7 +553,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       const float lv = row[e];
       v[i] = isnan(lv) ? -FLT_MAX : lv;   // a NaN logit ranks last
       const float b = bias ? fabsf(bias[e]) : 0.f;
-      const float r = (gamma * xn * wnorm[e] + ulast * (fabsf(v[i]) + b) + tiny) * 1.001f;
+      const float r = (gamma * xn * wnorm_of(e) + ulast * (fabsf(v[i]) + b) + tiny) * 1.001f;
       rmax = fmaxf(rmax, r);
       vmax = fmaxf(vmax, v[i]);
     }
@@ -583,7 +644,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       double d = fp64_logit(xrow, router_w + static_cast<size_t>(e) * H, H);
       const double b = bias ? static_cast<double>(bias[e]) : 0.0;
       d += b;
-      const double r = (gamma64 * xn * wnorm[e] + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
+      const double r = (gamma64 * xn * wnorm_of(e) + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
       r64 = fmax(r64, r);
       if (lane == 0) c_val[c] = d;
     }
@@ -662,20 +723,21 @@ static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
 }
 
 template <int kPer>
-static cudaError_t launch_topk(const RouterArgs& a, int acc64, int nchain, cudaStream_t st) {
+static cudaError_t launch_topk(const RouterArgs& a, int acc64, int nchain, int nsplit,
+                               cudaStream_t st) {
   return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
-                    a.xnorm, a.wnorm, a.bias, a.hidden, a.router_w, a.T, a.H, a.E, a.k, acc64,
-                    nchain, a.topk_ids, a.topk_w, a.cand, a.hdr);
+                    a.xnorm, a.wnorm, a.amax_tok, a.rsplit, nsplit, a.bias, a.hidden, a.router_w,
+                    a.T, a.H, a.E, a.k, acc64, nchain, a.topk_ids, a.topk_w, a.cand, a.hdr);
 }
 
-static cudaError_t launch_logits_tiled(const RouterArgs& a, cudaStream_t st) {
+static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStream_t st) {
   auto kern = router_logits_tiled_kernel;
   const int smem = 2 * (kLgT + kLgE) * kLgLd * 4;
   cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return err;
-  dim3 grid((a.T + kLgT - 1) / kLgT, (a.E + kLgE - 1) / kLgE);
+  dim3 grid((a.T + kLgT - 1) / kLgT, (a.E + kLgE - 1) / kLgE, nsplit);
   return launch_pdl(kern, grid, dim3(256), smem, st, a.hidden, a.router_w, a.bias, a.T, a.H, a.E,
-                    a.logits, a.xnorm, a.wnorm, a.amax_tok);
+                    a.logits, a.xnorm, a.wnorm, a.amax_tok, a.rsplit);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
@@ -684,9 +746,17 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   const bool acc64 = static_cast<double>(a.T) * a.E * a.H <= static_cast<double>(1 << 28);
   cudaError_t err;
   int nchain;
+  int nsplit = 1;
   if (!acc64 && a.E >= 32) {
-    // large batch: register-tiled fp32 GEMM (blocked summation, see above)
-    err = launch_logits_tiled(a, st);
+    // large batch: register-tiled fp32 GEMM (blocked summation, see above),
+    // split over K until the grid fills two CTAs per SM
+    const int tiles = ((a.T + kLgT - 1) / kLgT) * ((a.E + kLgE - 1) / kLgE);
+    if (a.rsplit != nullptr) {
+      const int want = (2 * current_sm_count() + tiles - 1) / tiles;
+      nsplit = want < 1 ? 1 : (want > kRouterSplits ? kRouterSplits : want);
+      if (nsplit > a.H / kLgK) nsplit = a.H / kLgK;
+    }
+    err = launch_logits_tiled(a, nsplit, st);
     nchain = a.H / kLgK + 64;
   } else {
     // tokens per CTA: the largest of 16, 8, 4, 2 that still gives two waves
@@ -713,9 +783,9 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   }
   if (err != cudaSuccess) return err;
   const int f64 = acc64 ? 1 : 0;
-  if (a.E <= 64) return launch_topk<2>(a, f64, nchain, st);
-  if (a.E <= 256) return launch_topk<8>(a, f64, nchain, st);
-  return launch_topk<kMaxExperts / 32>(a, f64, nchain, st);
+  if (a.E <= 64) return launch_topk<2>(a, f64, nchain, nsplit, st);
+  if (a.E <= 256) return launch_topk<8>(a, f64, nchain, nsplit, st);
+  return launch_topk<kMaxExperts / 32>(a, f64, nchain, nsplit, st);
 }
 
 }  // namespace moe

@@ -130,14 +130,17 @@ def test_route_bias_only(cuda_ok):
 # ------------------------------------------------------------------- align --
 @pytest.mark.parametrize("T,E,k,mode", [(1, 4, 1, "rand"), (37, 12, 3, "rand"), (64, 256, 8, "rand"),
                                         (4096, 128, 8, "rand"), (300, 40, 5, "hot"), (16, 1, 1, "rand"),
-                                        (513, 1000, 7, "rand")])
+                                        (513, 1000, 7, "rand"),
+                                        # T*k >= 8192: two grids over slices
+                                        (1024, 16, 8, "rand"), (1500, 1024, 7, "rand"),
+                                        (3001, 64, 6, "hot"), (262144, 3, 1, "rand")])
 def test_align_bit_exact(cuda_ok, T, E, k, mode):
     rng = np.random.default_rng(T * 7 + E)
     if mode == "hot":
         ids = np.stack([np.concatenate([[0], rng.choice(np.arange(1, E), k - 1, replace=False)])
                         for _ in range(T)])
-    else:
-        ids = np.stack([rng.choice(E, k, replace=False) for _ in range(T)])
+    else:   # k distinct experts per token
+        ids = np.argsort(rng.random((T, E)), axis=1)[:, :k]
     ids = ids.astype(np.int32)
     c, o, p, ip = layer.moe_align(torch.from_numpy(ids).cuda(), E)
     torch.cuda.synchronize()
@@ -148,9 +151,11 @@ def test_align_bit_exact(cuda_ok, T, E, k, mode):
     assert np.array_equal(ip.cpu().numpy(), rip)
 
 
-def test_align_rejects_bad_ids(cuda_ok):
-    ids = torch.tensor([[0, 5], [1, 2]], dtype=torch.int32, device="cuda")
-    ws = layer.make_workspace(2, 128, 4, 128, 2, 0)
+@pytest.mark.parametrize("T", [2, 5000])
+def test_align_rejects_bad_ids(cuda_ok, T):
+    ids = torch.randint(0, 4, (T, 2), dtype=torch.int32, device="cuda")
+    ids[0, 1] = 5
+    ws = layer.make_workspace(T, 128, 4, 128, 2, 0)
     layer.moe_align(ids, 4, workspace=ws)
     code, info = layer.get_status(ws)
     assert code == 6
