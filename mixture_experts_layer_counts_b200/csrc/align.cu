@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a, int mode, int 
 
   // tile schedule: swap-AB chunks of <= swap_chunk tokens for experts
   // with count <= swap_max_count, normal-orientation tiles of kNormalTokens
-  // tokens for the rest.
+  // tokens (down GEMM) and of kPairTokens tokens (gate/up GEMM) for the rest.
   const bool ex = threadIdx.x < E && c > 0;
   const bool sw = ex && c <= a.swap_max_count;
   const int nsw = sw ? (c + a.swap_chunk - 1) / a.swap_chunk : 0;
@@ -198,6 +198,10 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a, int mode, int 
   __syncthreads();
   const int ono = block_exclusive_scan(nno, tmp32, &total);
   const int tno = total;
+  __syncthreads();
+  const int npr = (ex && !sw) ? (c + kPairTokens - 1) / kPairTokens : 0;
+  const int opr = block_exclusive_scan(npr, tmp32, &total);
+  const int tpr = total;
   for (int i = 0; i < nsw; ++i) {
     const int n0 = i * a.swap_chunk;
     a.chunks_swap[osw + i] = make_int4(threadIdx.x, excl + n0, min(a.swap_chunk, c - n0), i);
@@ -206,9 +210,14 @@ __global__ void __launch_bounds__(1024) align_kernel(AlignArgs a, int mode, int 
     const int n0 = i * kNormalTokens;
     a.chunks_normal[ono + i] = make_int4(threadIdx.x, excl + n0, min(kNormalTokens, c - n0), i);
   }
+  for (int i = 0; i < npr; ++i) {
+    const int n0 = i * kPairTokens;
+    a.chunks_pair[opr + i] = make_int4(threadIdx.x, excl + n0, min(kPairTokens, c - n0), i);
+  }
   if (threadIdx.x == 0) {
     a.hdr[kHdrChunksSwap] = static_cast<uint32_t>(tsw);
     a.hdr[kHdrChunksNormal] = static_cast<uint32_t>(tno);
+    a.hdr[kHdrChunksPair] = static_cast<uint32_t>(tpr);
   }
 
   // FP8 activation scale: s1 = amax / 448 (one IEEE fp32 division); amax == 0 -> 1

@@ -208,6 +208,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
+               at<int4>(ws, L.chunks_pair),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
                at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots, at<int>(ws, L.slice_hist)};
   MOE_TRY(cuda_status(launch_align(aa, st)));
@@ -249,8 +250,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   }
   if (any_normal) {
     GemmArgs g = g13;
-    g.chunks = at<int4>(ws, L.chunks_normal);
-    g.nchunks = hdr + kHdrChunksNormal;
+    g.chunks = at<int4>(ws, L.chunks_pair);
+    g.nchunks = hdr + kHdrChunksPair;
     g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
     g.amax_cta = amax_cta + (any_swap ? grid : 0);
     g.flags = flags + 1 * kMaxSlots;
@@ -388,6 +389,7 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t
     return MOE_ERR_WORKSPACE_TOO_SMALL;
   AlignArgs aa{topk_ids, T, E, top_k, counts, offsets, perm, inv_perm,
                at<int4>(workspace, L.chunks_swap), at<int4>(workspace, L.chunks_normal),
+               at<int4>(workspace, L.chunks_pair),
                swap_threshold(), gemm_swap_chunk(), nullptr, at<uint32_t>(workspace, L.header),
                at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots,
                at<int>(workspace, L.slice_hist)};

@@ -32,6 +32,7 @@ constexpr int kTileM = 128;            // rows of the A operand per MMA (M)
 constexpr int kSwapMaxTokens = 64;     // largest token chunk in swap-AB (N <= 64)
 constexpr int kTokenBox = 16;          // rows per TMA box of the token operand (swap-AB)
 constexpr int kNormalTokens = 128;     // token rows per tile in normal orientation (M)
+constexpr int kPairTokens = 256;       // gate/up GEMM, normal orientation: two M tiles per weight tile
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxGrid = 1024;          // persistent grids never exceed this
@@ -45,6 +46,7 @@ constexpr int kHdrInfo = 1;            // where it happened
 constexpr int kHdrChunksSwap = 4;      // number of swap-AB token chunks
 constexpr int kHdrChunksNormal = 5;    // number of normal-orientation token tiles
 constexpr int kHdrUncertain = 6;       // tokens whose router ordering needed fp64 / exact
+constexpr int kHdrChunksPair = 7;      // number of normal-orientation 256-token chunks (gate/up GEMM)
 constexpr int kHdrScaleS1 = 8;         // fp32 bits: activation scale (FP8)
 constexpr int kHdrScaleS2 = 9;         // fp32 bits: intermediate scale (FP8)
 constexpr int kHdrBarrier = 12;        // grid barrier counter
@@ -60,9 +62,9 @@ __device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, u
 struct Layout {
   size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand, rsplit;
   size_t slice_hist;
-  size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, gemm_flags, partials;
+  size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, chunks_pair, gemm_flags, partials;
   size_t xperm, inter, h32, ysc, staging_in, staging_out, total;
-  int max_chunks_swap, max_chunks_normal;
+  int max_chunks_swap, max_chunks_normal, max_chunks_pair;
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -106,6 +108,8 @@ inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   L.max_chunks_normal = static_cast<int>(E + A / kNormalTokens + 1);
   L.chunks_swap = take(static_cast<size_t>(L.max_chunks_swap) * 16);
   L.chunks_normal = take(static_cast<size_t>(L.max_chunks_normal) * 16);
+  L.max_chunks_pair = static_cast<int>(E + A / kPairTokens + 1);
+  L.chunks_pair = take(static_cast<size_t>(L.max_chunks_pair) * 16);
   L.gemm_flags = take(static_cast<size_t>(kGemmLaunches) * kMaxSlots * 4);
   L.partials = take(static_cast<size_t>(kMaxSlots) * kPartialSlotFloats * 4);
   const size_t eb = fp8 ? 1 : 2;

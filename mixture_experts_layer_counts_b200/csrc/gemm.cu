@@ -60,11 +60,17 @@ template <Orient O, Proj P, bool FP8, int KA, int BNT>
 struct Cfg {
   static constexpr bool kSwap = O == Orient::kSwap;
   static constexpr bool kDual = P == Proj::kW13;
+  // normal-orientation gate/up GEMM: a unit is a 256-token chunk (two M
+  // tiles) x one weight tile, so each weight byte staged feeds two MMAs
+  static constexpr bool kPair = !kSwap && kDual;
+  static constexpr int kChunkTokens = kPair ? kPairTokens : kNormalTokens;
   static constexpr int kBN = kSwap ? BNT : (kDual ? 128 : 256);   // max N
   static constexpr int kATile = kTileM * kAtomBytes;
   static constexpr int kBTile = kBN * kAtomBytes;
-  static constexpr int kNumA = (kSwap && kDual) ? 2 : 1;
+  // swap-AB w13: A = gate and up weight tiles; pair: A = the two token tiles
+  static constexpr int kNumA = ((kSwap && kDual) || kPair) ? 2 : 1;
   static constexpr int kNumB = (!kSwap && kDual) ? 2 : 1;
+  static constexpr int kBOff = kNumA * kATile;                        // B within an atom set
   static constexpr int kAtomSet = kNumA * kATile + kNumB * kBTile;   // one K atom of every operand
   static constexpr int kStageBytes = KA * kAtomSet;
   // epilogue warps: 4 (one per TMEM lane quadrant); the normal orientation
@@ -79,8 +85,9 @@ struct Cfg {
   static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kNumAcc = kDual ? 2 : 1;
-  static constexpr int kAccCols = kNumAcc * kBN;               // per TMEM buffer
-  static constexpr int kTmemCols = 2 * kAccCols;               // 128, 256 or 512
+  static constexpr int kAccCols = kNumAcc * kBN * (kPair ? 2 : 1);   // per TMEM buffer
+  static constexpr int kAccBufs = kPair ? 1 : 2;               // pair: 512 columns, one buffer
+  static constexpr int kTmemCols = kAccBufs * kAccCols;        // 128, 256 or 512
   static constexpr int kSmemBytes =
       kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes;
   static constexpr int kAtomElems = FP8 ? 128 : 64;
@@ -135,8 +142,8 @@ struct Segments {
 // the token chunks that share a weight tile are consecutive units; dealt
 // round-robin, they run on neighbouring CTAs at the same time and share one
 // DRAM fetch of that tile through L2.  chunk.w = index of the chunk inside its
-// expert; the expert has ceil(counts[e] / kNormalTokens) chunks.
-template <bool kGrouped>
+// expert; the expert has ceil(counts[e] / kChunkTokens) chunks.
+template <bool kGrouped, int kChunkTokens>
 __device__ __forceinline__ void unit_coords(const GemmArgs& a, int u, int4& ch, int& mt) {
   const int cs = u / a.mtiles;   // a chunk of the unit's expert
   if constexpr (!kGrouped) {
@@ -145,7 +152,7 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& a, int u, int4& ch, 
   } else {
     const int4 s = a.chunks[cs];
     const int c0 = cs - s.w;   // the expert's first chunk
-    const int nch = (a.counts[s.x] + kNormalTokens - 1) / kNormalTokens;
+    const int nch = (a.counts[s.x] + kChunkTokens - 1) / kChunkTokens;
     const int local = u - c0 * a.mtiles;
     mt = local / nch;
     ch = a.chunks[c0 + (local - mt * nch)];
@@ -277,7 +284,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     auto issue = [&](int stage, int u, int kb, bool first, int parts) {
       int4 ch;
       int mt;
-      unit_coords<kRR>(a, u, ch, mt);
+      unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const int wrow0 = e * a.w_rows_per_expert + mt * (C::kSwap ? kTileM : C::kBN);
       const int nbox = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox : 0;
@@ -298,11 +305,15 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
               tma_load_2d(sb + q * kTokenBox * kAtomBytes, &tm_x, &full[stage], kc, p0 + q * kTokenBox, pol_x);
           }
         } else {
-          if (parts & 2) tma_load_2d(sa, &tm_x, &full[stage], kc, p0, pol_x);
+          if (parts & 2) {
+            tma_load_2d(sa, &tm_x, &full[stage], kc, p0, pol_x);
+            if constexpr (C::kPair)   // second M tile only when the chunk has one
+              if (nv > kTileM) tma_load_2d(sa + C::kATile, &tm_x, &full[stage], kc, p0 + kTileM, pol_x);
+          }
           if (parts & 1) {
-            tma_load_2d(sa + C::kATile, &tm_w, &full[stage], kc, wrow0, pol_w);
+            tma_load_2d(sa + C::kBOff, &tm_w, &full[stage], kc, wrow0, pol_w);
             if constexpr (C::kDual)
-              tma_load_2d(sa + C::kATile + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
+              tma_load_2d(sa + C::kBOff + C::kBTile, &tm_w, &full[stage], kc, wrow0 + a.up_offset, pol_w);
           }
         }
       }
@@ -311,9 +322,14 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       if constexpr (C::kSwap) {
         int4 ch;
         int mt;
-        unit_coords<kRR>(a, u, ch, mt);
+        unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
         const int nvpad = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
         return KA * (C::kNumA * C::kATile + nvpad * kAtomBytes);
+      } else if constexpr (C::kPair) {
+        int4 ch;
+        int mt;
+        unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
+        return ch.z > kTileM ? C::kStageBytes : C::kStageBytes - KA * C::kATile;
       } else {
         return C::kStageBytes;
       }
@@ -382,8 +398,8 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     Segments seg = seg0;
     int u, kb0, kb1;
     while (ok && seg.next(u, kb0, kb1)) {
-      const int buf = it & 1;
-      const uint32_t accph = (it >> 1) & 1;
+      const int buf = it % C::kAccBufs;
+      const uint32_t accph = (it / C::kAccBufs) & 1;
       ++it;
       if (!mbar_wait(&acc_empty[buf], accph ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty, a.timeout_ns)) {
         ok = false;
@@ -392,7 +408,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       tc_fence_after();
       int4 ch;
       int mt;
-      unit_coords<kRR>(a, u, ch, mt);
+      unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       int n;
       if constexpr (C::kSwap) {
         n = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
@@ -422,8 +438,13 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
           } else {
             // w13: the gate and up tiles are adjacent in smem, so one MMA with
             // N = 2 * kBN covers both; its columns [0, kBN) are the gate
-            // accumulator and [kBN, 2 kBN) the up accumulator (d1 = d0 + kBN)
-            mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(st + C::kATile + off), idesc, acc);
+            // accumulator and [kBN, 2 kBN) the up accumulator.  Pair: the
+            // second token tile accumulates into the next 2 * kBN columns.
+            mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(st + C::kBOff + off), idesc, acc);
+            if constexpr (C::kPair)
+              if (ch.z > kTileM)
+                mma_ss<FP8>(d0 + 2 * C::kBN, sdesc_sw128(st + C::kATile + off),
+                            sdesc_sw128(st + C::kBOff + off), idesc, acc);
           }
         }
         issued = true;
@@ -449,14 +470,14 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     Segments seg = seg0;
     int u, kb0, kb1;
     while (seg.next(u, kb0, kb1)) {
-      const int buf = it & 1;
-      const uint32_t accph = (it >> 1) & 1;
+      const int buf = it % C::kAccBufs;
+      const uint32_t accph = (it / C::kAccBufs) & 1;
       ++it;
       if (!mbar_wait(&acc_full[buf], accph, abort_flag, a.hdr, kSiteEpiAccFull, a.timeout_ns)) break;
       tc_fence_after();
       int4 ch;
       int mt;
-      unit_coords<kRR>(a, u, ch, mt);
+      unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
       const int ncols = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox * kTokenBox : C::kBN;
@@ -555,18 +576,20 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
           }
         }
       } else if constexpr (C::kDual) {
-        // normal w13: h for token rows p0 + rb.., intermediate columns
-        // i0 + c0..  Warp half hx takes columns [hx kBN/2, (hx+1) kBN/2) of
-        // the gate and up accumulators.  Each 16-column piece of the warp's
-        // 32 rows is staged in smem, then written as whole row segments
-        // (bf16: 32 B, fp32: 64 B) with coalesced stores.
+        // normal w13 (pair): warp half hx takes token rows hx*128 + q*32 +
+        // lane of the 256-token chunk, whose gate and up accumulators sit at
+        // columns hx*2*kBN + [0, kBN) and + [kBN, 2 kBN).  Each 16-column
+        // piece of the warp's 32 rows is staged in smem, then written as
+        // whole row segments (bf16: 32 B, fp32: 64 B) with coalesced stores.
         float* sw = epi + (warp - 2) * 32 * C::kEpiLd;
         const int i0 = mt * C::kBN;
-        const int rb = q * 32;
         const int hx = (warp - 2) >> 2;
-        for (int c0 = hx * (C::kBN / 2); c0 < (hx + 1) * (C::kBN / 2); c0 += C::kEpiCols) {
+        const int rb = hx * kTileM + q * 32;   // first chunk row of this warp's block
+        const bool my_valid = rb + lane < nv;
+        const uint32_t th = tbase + hx * 2 * C::kBN;
+        for (int c0 = 0; c0 < (rb < nv ? C::kBN : 0); c0 += C::kEpiCols) {
           float v[2][16];
-          tmem_ld16x2_wait(tbase + c0, tbase + C::kBN + c0, v[0], v[1]);
+          tmem_ld16x2_wait(th + c0, th + C::kBN + c0, v[0], v[1]);
           float h[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -574,7 +597,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
             h[j] = __fdividef(gg, 1.0f + __expf(-gg)) * uv;
           }
           if constexpr (FP8) {
-            if (row < nv) {
+            if (my_valid) {
 #pragma unroll
               for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(h[j]));
             }

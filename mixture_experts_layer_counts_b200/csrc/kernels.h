@@ -70,6 +70,7 @@ struct AlignArgs {
   int32_t* inv_perm;
   int4* chunks_swap;
   int4* chunks_normal;
+  int4* chunks_pair;      // normal orientation, 256-token chunks (gate/up GEMM)
   int swap_max_count;     // experts with count <= this run swap-AB
   int swap_chunk;         // tokens per swap-AB chunk (the swap kernels' largest N)
   const float* amax_tok;  // FP8: per-token amax|x| (NULL on bf16)

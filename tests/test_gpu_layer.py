@@ -175,7 +175,8 @@ def test_forward_parity_bf16(cuda_ok, name):
 
 
 @pytest.mark.parametrize("force", [1, 2])
-@pytest.mark.parametrize("shape", [(37, 512, 12, 256, 3), (130, 256, 6, 384, 2), (200, 768, 8, 128, 8)])
+@pytest.mark.parametrize("shape", [(37, 512, 12, 256, 3), (130, 256, 6, 384, 2), (200, 768, 8, 128, 8),
+                                   (700, 256, 3, 256, 2)])
 def test_forward_forced_orientation(cuda_ok, force, shape):
     T, H, E, I, k = shape
     inp = custom_inputs(T, H, E, I, k, seed=sum(shape) + force, bias=True)
@@ -215,7 +216,9 @@ def test_forward_edge_shapes(cuda_ok, shape):
 
 
 @pytest.mark.parametrize("shape,force", [((16, 512, 8, 256, 2), 0), ((200, 512, 8, 256, 4), 2),
-                                         ((64, 1024, 16, 512, 8), 0)])
+                                         ((64, 1024, 16, 512, 8), 0),
+                                         # normal orientation, both token tiles of 256-token chunks
+                                         ((300, 256, 4, 384, 3), 2)])
 def test_forward_fp8_small(cuda_ok, shape, force):
     T, H, E, I, k = shape
     inp = custom_inputs(T, H, E, I, k, seed=5, fp8=True)
