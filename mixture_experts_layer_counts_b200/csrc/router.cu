@@ -174,14 +174,21 @@ __device__ double fp64_logit(const __nv_bfloat16* __restrict__ x, const __nv_bfl
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Kernel 1: logits[t, e] = sum_h x[t,h] w[e,h] + b[e], accumulated in fp64
-// (F64, decode-sized calls: the error bound then shrinks to the fp32 rounding
-// of the stored logit) or fp32 (large calls), stored as fp32; plus ||x_t||,
+// Kernel 1: logits[t, e] = sum_h x[t,h] w[e,h] + b[e], stored as fp32.
+// ACC = kAcc64: every product accumulated in fp64 (the smallest decode
+// calls; the bound is then the fp64 chain plus the final fp32 rounding).
+// ACC = kAccMixed: the 8 exact products of each 16-byte vector pair are summed
+// by an fp32 FMA chain (7 roundings) and the vector sums accumulated in fp64,
+// one fp64 conversion per 8 products instead of two per product (larger
+// decode calls, where conversions would dominate); bound 7 fp32 ulps of
+// sum|x w| plus the fp64 chain.  ACC = kAcc32: plain fp32 chains.  Plus ||x_t||,
 // ||w_e|| for the error bound and per-token amax|x| for the FP8 activation
 // scale.  CTA = TT tokens x 8 experts (one expert per warp), hidden rows
 // staged in smem, four 16-byte router-row loads in flight per lane.
 // ---------------------------------------------------------------------------
-template <int TT, bool F64>
+constexpr int kAcc32 = 0, kAcc64 = 1, kAccMixed = 2;
+
+template <int TT, int ACC>
 __global__ void __launch_bounds__(256) router_logits_kernel(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
@@ -246,6 +253,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
   }
 
   if (!has_e) return;
+  constexpr bool F64 = ACC != kAcc32;
   using Acc = typename std::conditional<F64, double, float>::type;
   Acc acc[TT];
 #pragma unroll
@@ -271,12 +279,18 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
       for (int tt = 0; tt < TT; ++tt) {
         float xf[8];
         unpack8(sx[tt * vpr + c], xf);
+        if constexpr (ACC == kAccMixed) {
+          float p = xf[0] * wf[0];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if constexpr (F64)
+          for (int i = 1; i < 8; ++i) p = fmaf(xf[i], wf[i], p);
+          acc[tt] += static_cast<double>(p);
+        } else if constexpr (ACC == kAcc64) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
             acc[tt] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[tt]);
-          else
-            acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[tt] = fmaf(xf[i], wf[i], acc[tt]);
         }
       }
     }
@@ -481,9 +495,9 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
 // Kernel 2: one warp per token.  fp32 softmax, top-(k+1) by repeated warp
 // argmax, certification against the error bound, fallback tiers 2-3.
 // kPer = experts per lane (register arrays sized by the expert count).
-// acc64: the logits were accumulated in fp64 and rounded once to fp32, so
-// the bound is the fp64 summation term plus the fp32 half-ulp of the stored
-// value; otherwise the fp32 summation bound applies.
+// gamma: relative summation bound of the logit kernel that ran (times
+// sum|x w| <= ||x|| ||w||); ulast: relative error of the last roundings (bias
+// add, storage to fp32).
 // nsplit > 1: the logits kernel ran split-K; this kernel first adds the
 // token's nsplit partial logits in split order, then the bias, stores the
 // row to `logits`, and forms ||x_t||, amax|x_t| and ||w_e|| from the partial
@@ -494,7 +508,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     float* __restrict__ logits, float* __restrict__ xnorm, const float* __restrict__ wnorm,
     float* __restrict__ amax_tok, const float* __restrict__ rsplit, int nsplit,
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
-    const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, int acc64, int nchain,
+    const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
     uint32_t* __restrict__ hdr) {
   pdl_wait();
@@ -534,12 +548,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     for (int z = 0; z < nsplit; ++z) ss += p_wss[static_cast<size_t>(z) * E + e];
     return sqrtf(ss);
   };
-  // gamma_n for the summation chain (n = nchain, the logit kernel's longest
-  // chain of roundings), the relative error of the last roundings (bias add,
-  // storage to fp32), and H products that might underflow (2^-149 each)
-  const float gamma = acc64 ? static_cast<float>(nchain * 1.1102230246251565e-16 * 1.0001)
-                            : static_cast<float>(nchain) * 5.9604645e-08f * 1.0001f;
-  const float ulast = acc64 ? 5.9604645e-08f : 1.1920929e-07f;
+  // plus H products that might underflow in fp32 (2^-149 each)
   const float tiny = static_cast<float>(H) * 1.4012985e-45f;
 
   float v[kPer];
@@ -711,9 +720,9 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 }
 
 // ---------------------------------------------------------------------------
-template <int TT, bool F64>
+template <int TT, int ACC>
 static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
-  auto kern = router_logits_kernel<TT, F64>;
+  auto kern = router_logits_kernel<TT, ACC>;
   const int smem = TT * a.H * 2;
   cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
   if (err != cudaSuccess) return err;
@@ -723,11 +732,11 @@ static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
 }
 
 template <int kPer>
-static cudaError_t launch_topk(const RouterArgs& a, int acc64, int nchain, int nsplit,
+static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, int nsplit,
                                cudaStream_t st) {
   return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
                     a.xnorm, a.wnorm, a.amax_tok, a.rsplit, nsplit, a.bias, a.hidden, a.router_w,
-                    a.T, a.H, a.E, a.k, acc64, nchain, a.topk_ids, a.topk_w, a.cand, a.hdr);
+                    a.T, a.H, a.E, a.k, gamma, ulast, a.topk_ids, a.topk_w, a.cand, a.hdr);
 }
 
 static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStream_t st) {
@@ -743,7 +752,12 @@ static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStre
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   // fp64 accumulation while the logit work is small (decode batches); fp32
   // with the wider certified bound for large batches
-  const bool acc64 = static_cast<double>(a.T) * a.E * a.H <= static_cast<double>(1 << 28);
+  // fp64 accumulation while the logit work is small (decode batches): per
+  // product up to 2^25 multiply-adds, in 8-product fp32 blocks up to 2^28;
+  // fp32 with the wider certified bound for large batches
+  const double macs = static_cast<double>(a.T) * a.E * a.H;
+  const bool acc64 = macs <= static_cast<double>(1 << 28);
+  const int mode = !acc64 ? kAcc32 : (macs <= static_cast<double>(1 << 25) ? kAcc64 : kAccMixed);
   cudaError_t err;
   int nchain;
   int nsplit = 1;
@@ -772,20 +786,37 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
         break;
       }
     }
-    switch (tt) {
-      case 16: err = acc64 ? launch_logits<16, true>(a, st) : launch_logits<16, false>(a, st); break;
-      case 8: err = acc64 ? launch_logits<8, true>(a, st) : launch_logits<8, false>(a, st); break;
-      case 4: err = acc64 ? launch_logits<4, true>(a, st) : launch_logits<4, false>(a, st); break;
-      case 2: err = acc64 ? launch_logits<2, true>(a, st) : launch_logits<2, false>(a, st); break;
-      default: err = acc64 ? launch_logits<1, true>(a, st) : launch_logits<1, false>(a, st); break;
+    switch (mode * 32 + tt) {
+      case kAcc64 * 32 + 16: err = launch_logits<16, kAcc64>(a, st); break;
+      case kAcc64 * 32 + 8: err = launch_logits<8, kAcc64>(a, st); break;
+      case kAcc64 * 32 + 4: err = launch_logits<4, kAcc64>(a, st); break;
+      case kAcc64 * 32 + 2: err = launch_logits<2, kAcc64>(a, st); break;
+      case kAcc64 * 32 + 1: err = launch_logits<1, kAcc64>(a, st); break;
+      case kAccMixed * 32 + 16: err = launch_logits<16, kAccMixed>(a, st); break;
+      case kAccMixed * 32 + 8: err = launch_logits<8, kAccMixed>(a, st); break;
+      case kAccMixed * 32 + 4: err = launch_logits<4, kAccMixed>(a, st); break;
+      case kAccMixed * 32 + 2: err = launch_logits<2, kAccMixed>(a, st); break;
+      case kAccMixed * 32 + 1: err = launch_logits<1, kAccMixed>(a, st); break;
+      case kAcc32 * 32 + 16: err = launch_logits<16, kAcc32>(a, st); break;
+      case kAcc32 * 32 + 8: err = launch_logits<8, kAcc32>(a, st); break;
+      case kAcc32 * 32 + 4: err = launch_logits<4, kAcc32>(a, st); break;
+      case kAcc32 * 32 + 2: err = launch_logits<2, kAcc32>(a, st); break;
+      default: err = launch_logits<1, kAcc32>(a, st); break;
     }
     nchain = a.H / 32 + 16;
   }
   if (err != cudaSuccess) return err;
-  const int f64 = acc64 ? 1 : 0;
-  if (a.E <= 64) return launch_topk<2>(a, f64, nchain, nsplit, st);
-  if (a.E <= 256) return launch_topk<8>(a, f64, nchain, nsplit, st);
-  return launch_topk<kMaxExperts / 32>(a, f64, nchain, nsplit, st);
+  // relative bounds (unit roundoff u32 = 2^-24, u64 = 2^-53): an fp64 chain
+  // of nchain roundings; the mixed form adds a 7-step fp32 chain per 8
+  // products; fp32 chains of nchain roundings
+  const double u32 = 5.9604644775390625e-08, u64 = 1.1102230246251565e-16;
+  const float gamma = mode == kAcc64     ? static_cast<float>(nchain * u64 * 1.0001)
+                      : mode == kAccMixed ? static_cast<float>((7.0 * u32 + nchain * u64) * 1.0001)
+                                          : static_cast<float>(nchain * u32 * 1.0001);
+  const float ulast = acc64 ? static_cast<float>(u32) : static_cast<float>(2.0 * u32);
+  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, nsplit, st);
+  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, nsplit, st);
+  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, nsplit, st);
 }
 
 }  // namespace moe

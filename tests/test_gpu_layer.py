@@ -66,6 +66,20 @@ def _route_pair(x, wr, k, bias=None):
 def test_route_large_batch_tiled(cuda_ok, T, H, E, k, bias, dup):
     # T * E * H > 2^28 with E >= 32: logits from the register-tiled fp32 kernel
     assert T * E * H > 2 ** 28 and E >= 32
+    _route_case(T, H, E, k, bias, dup)
+
+
+@pytest.mark.parametrize("T,H,E,k,bias,dup", [
+    (300, 4096, 64, 8, True, True),       # ties, 8-product fp32 blocks accumulated in fp64
+    (70, 7168, 96, 6, False, False),
+])
+def test_route_mixed_accumulation(cuda_ok, T, H, E, k, bias, dup):
+    # 2^25 < T * E * H <= 2^28: the decode logits kernel in its mixed form
+    assert 2 ** 25 < T * E * H <= 2 ** 28
+    _route_case(T, H, E, k, bias, dup)
+
+
+def _route_case(T, H, E, k, bias, dup):
     rng = np.random.default_rng(T + H + E)
     x = rng.standard_normal((T, H))
     wr = rng.standard_normal((E, H)) * 0.05
