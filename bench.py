@@ -126,14 +126,18 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
+    """(rank, world, local rank) from the launcher's environment; one process
+    per GPU over NCCL, or gloo on a host without GPUs (the CPU tests)."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         import datetime
 
-        torch.cuda.set_device(local)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -145,11 +149,29 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """Max of a per-rank float over all ranks (every rank gets it)."""
     if world == 1:
         return v
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_inputs(wl, dev, rank, world):
+    """Each rank serves its own batch: rank-dependent hidden states, the same
+    weights (same seed) on every rank."""
+    inp = make_inputs(wl, dev, seed=wl["seed"])
+    if world > 1:
+        from mixture_experts_layer_counts_b200.inputs import make_hidden
+
+        inp["hidden"] = make_hidden(wl, dev, seed=wl["seed"] + 1000 * rank)
+    return inp
+
+
+def whole_job_tokens_per_s(world, T, steps, max_total_ms):
+    """Tokens all ranks processed / the slowest rank's device time."""
+    return world * T * steps / (max_total_ms * 1e-3)
 
 
 def oracle_sample_seconds(inp_host, wl, tokens):
@@ -230,12 +252,7 @@ def run_ours(args, wl, rank, world, local):
 
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
-    # each rank serves its own decode batch: rank-dependent hidden, shared weight seed
-    inp = make_inputs(wl, dev, seed=wl["seed"])
-    if world > 1:
-        from mixture_experts_layer_counts_b200.inputs import make_hidden
-
-        inp["hidden"] = make_hidden(wl, dev, seed=wl["seed"] + 1000 * rank)
+    inp = rank_inputs(wl, dev, rank, world)
     T, H, E, I, k = inp["T"], inp["H"], inp["E"], inp["I"], inp["top_k"]
     dt = layer.dtype_code(inp["w13"])
     ws = layer.make_workspace(T, H, E, I, k, dt, dev)
@@ -301,7 +318,7 @@ def run_ours(args, wl, rank, world, local):
     step_ms = [a_.elapsed_time(b_) for a_, b_ in tev]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms * 1e-3)
+    value = whole_job_tokens_per_s(world, T, args.steps, total_ms)
     del graph
 
     # Per-kernel breakdown: the same graph with the library's 8 stage events

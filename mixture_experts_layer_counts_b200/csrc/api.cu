@@ -202,15 +202,14 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
                 at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit)};
-  MOE_TRY(cuda_status(launch_router(ra, st)));
-  record(dbg, 1, st);
-
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
                at<int4>(ws, L.chunks_pair),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
                at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots, at<int>(ws, L.slice_hist)};
+  MOE_TRY(cuda_status(launch_router(ra, st)));
+  record(dbg, 1, st);
   MOE_TRY(cuda_status(launch_align(aa, st)));
   record(dbg, 2, st);
 

@@ -188,24 +188,23 @@ __device__ double fp64_logit(const __nv_bfloat16* __restrict__ x, const __nv_bfl
 // ---------------------------------------------------------------------------
 constexpr int kAcc32 = 0, kAcc64 = 1, kAccMixed = 2;
 
+// The CTA body (warps 0..7 compute; any further warps only help staging).
 template <int TT, int ACC>
-__global__ void __launch_bounds__(256) router_logits_kernel(
+__device__ __forceinline__ void logits_body(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
-    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
-  extern __shared__ uint4 sx[];
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok, uint4* sx) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
   const int t0 = blockIdx.x * TT;
   const int nt = min(TT, T - t0);
   const int vpr = H / 8;   // 16-byte vectors per row
   const uint4* hv = reinterpret_cast<const uint4*>(hidden);
   const int e = blockIdx.y * 8 + warp;
-  const bool has_e = e < E;
+  const bool has_e = warp < 8 && e < E;
   const uint4* wrow = reinterpret_cast<const uint4*>(router_w) + static_cast<size_t>(has_e ? e : 0) * vpr;
   constexpr int U = 8;     // 16-byte router-row loads in flight per lane
 
-  pdl_wait();
-  pdl_launch_next();
   // the first U vectors of this warp's router row are requested before the
   // token rows are staged, so both sets of loads are in flight together
   uint4 wv[U];
@@ -232,7 +231,7 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
   __syncthreads();
 
   if (blockIdx.y == 0) {
-    for (int r = warp; r < nt; r += 8) {
+    for (int r = warp; r < nt; r += nwarps) {
       float ss = 0.f, am = 0.f;
       for (int c = lane; c < vpr; c += 32) {
         float f[8];
@@ -309,6 +308,17 @@ __global__ void __launch_bounds__(256) router_logits_kernel(
       logits[static_cast<size_t>(t0 + tt) * E + e] = static_cast<float>(acc[tt] + static_cast<Acc>(b));
     if (blockIdx.x == 0) wnorm[e] = sqrtf(wsq);
   }
+}
+
+template <int TT, int ACC>
+__global__ void __launch_bounds__(256) router_logits_kernel(
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
+    const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
+  extern __shared__ uint4 sx[];
+  pdl_wait();
+  pdl_launch_next();
+  logits_body<TT, ACC>(hidden, router_w, bias, T, H, E, logits, xnorm, wnorm, amax_tok, sx);
 }
 
 // ---------------------------------------------------------------------------
@@ -503,19 +513,17 @@ __global__ void __launch_bounds__(256) router_logits_tiled_kernel(
 // row to `logits`, and forms ||x_t||, amax|x_t| and ||w_e|| from the partial
 // sums.
 // ---------------------------------------------------------------------------
+// Top-k of token t by the calling warp.  Logits, norms and partials are
+// read through L2 (they may come from other CTAs of the same grid).
 template <int kPer>
-__global__ void __launch_bounds__(256) router_topk_kernel(
-    float* __restrict__ logits, float* __restrict__ xnorm, const float* __restrict__ wnorm,
+__device__ void topk_token(
+    int t, float* __restrict__ logits, float* __restrict__ xnorm, const float* __restrict__ wnorm,
     float* __restrict__ amax_tok, const float* __restrict__ rsplit, int nsplit,
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
     uint32_t* __restrict__ hdr) {
-  pdl_wait();
-  pdl_launch_next();
   const int lane = threadIdx.x & 31;
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
   const int nper = (E + 31) / 32;
   float* row = logits + static_cast<size_t>(t) * E;
   const float* p_xss = rsplit + static_cast<size_t>(nsplit) * T * E;
@@ -525,8 +533,8 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   if (nsplit > 1) {
     float ss = 0.f, am = 0.f;
     for (int z = 0; z < nsplit; ++z) {
-      ss += p_xss[static_cast<size_t>(z) * T + t];
-      am = fmaxf(am, p_xam[static_cast<size_t>(z) * T + t]);
+      ss += __ldcg(p_xss + static_cast<size_t>(z) * T + t);
+      am = fmaxf(am, __ldcg(p_xam + static_cast<size_t>(z) * T + t));
     }
     xn = sqrtf(ss);
     if (lane == 0) {
@@ -534,18 +542,18 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
       amax_tok[t] = am;
     }
     for (int e = lane; e < E; e += 32) {
-      float v = rsplit[static_cast<size_t>(t) * E + e];
-      for (int z = 1; z < nsplit; ++z) v += rsplit[(static_cast<size_t>(z) * T + t) * E + e];
+      float v = __ldcg(rsplit + static_cast<size_t>(t) * E + e);
+      for (int z = 1; z < nsplit; ++z) v += __ldcg(rsplit + (static_cast<size_t>(z) * T + t) * E + e);
       row[e] = v + (bias ? bias[e] : 0.f);
     }
     __syncwarp();
   } else {
-    xn = xnorm[t];
+    xn = __ldcg(xnorm + t);
   }
   auto wnorm_of = [&](int e) -> float {
-    if (nsplit <= 1) return wnorm[e];
+    if (nsplit <= 1) return __ldcg(wnorm + e);
     float ss = 0.f;
-    for (int z = 0; z < nsplit; ++z) ss += p_wss[static_cast<size_t>(z) * E + e];
+    for (int z = 0; z < nsplit; ++z) ss += __ldcg(p_wss + static_cast<size_t>(z) * E + e);
     return sqrtf(ss);
   };
   // plus H products that might underflow in fp32 (2^-149 each)
@@ -559,7 +567,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const int e = lane + 32 * i;
     v[i] = -FLT_MAX;
     if (i < nper && e < E) {
-      const float lv = row[e];
+      const float lv = __ldcg(row + e);
       v[i] = isnan(lv) ? -FLT_MAX : lv;   // a NaN logit ranks last
       const float b = bias ? fabsf(bias[e]) : 0.f;
       const float r = (gamma * xn * wnorm_of(e) + ulast * (fabsf(v[i]) + b) + tiny) * 1.001f;
@@ -626,7 +634,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     auto put = [&](int e) {   // slot `got` takes expert e
       if (lane == got) {
         my_idx = e;
-        const float lv = row[e];
+        const float lv = __ldcg(row + e);
         my_v = isnan(lv) ? -FLT_MAX : lv;
       }
       ++got;
@@ -717,6 +725,22 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     topk_ids[static_cast<size_t>(t) * k + lane] = my_idx;
     topk_w[static_cast<size_t>(t) * k + lane] = p / psum;
   }
+}
+
+template <int kPer>
+__global__ void __launch_bounds__(256) router_topk_kernel(
+    float* __restrict__ logits, float* __restrict__ xnorm, const float* __restrict__ wnorm,
+    float* __restrict__ amax_tok, const float* __restrict__ rsplit, int nsplit,
+    const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
+    const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
+    int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
+    uint32_t* __restrict__ hdr) {
+  pdl_wait();
+  pdl_launch_next();
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  topk_token<kPer>(t, logits, xnorm, wnorm, amax_tok, rsplit, nsplit, bias, hidden, router_w, T, H,
+                   E, k, gamma, ulast, topk_ids, topk_w, cand, hdr);
 }
 
 // ---------------------------------------------------------------------------
