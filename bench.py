@@ -259,6 +259,8 @@ def run_ours(args, wl, rank, world, local):
     out = torch.empty((T, H), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     fwd = dict(w13_scale=inp["w13_scale"], w2_scale=inp["w2_scale"], out=out, workspace=ws)
+    if args.batch_invariant:
+        fwd["batch_invariant"] = True
 
     def step(events=None):
         layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
@@ -379,11 +381,18 @@ def run_ours(args, wl, rank, world, local):
     e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
     barrier(world)
     torch.cuda.synchronize()
+    dev_hidden = torch.empty_like(inp["hidden"])
     for i in range(e2e_steps):
         flush.zero_()
         e_ev[i][0].record(stream)
-        layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k, hout, ws,
-                                 inp["w13_scale"], inp["w2_scale"])
+        if args.batch_invariant:   # no host-I/O entry point: the same copies around the call
+            dev_hidden.copy_(hin, non_blocking=True)
+            layer.moe_forward(dev_hidden, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                              **fwd)
+            hout.copy_(out, non_blocking=True)
+        else:
+            layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                                     hout, ws, inp["w13_scale"], inp["w2_scale"])
         e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -424,7 +433,8 @@ def run_ours(args, wl, rank, world, local):
         "dtype": "fp8-e4m3" if dt == 1 else "bf16", "data": "synthetic",
         "config": {"workload": f"{args.workload}: {describe(wl)}", "global_batch": world * T,
                    "active_experts": e_act, "l2": "flushed (256 MiB write) between timed steps",
-                   "parallelism": f"dp{world} (independent decode batches)"},
+                   "parallelism": f"dp{world} (independent decode batches)",
+                   "mode": "batch_invariant" if args.batch_invariant else "default"},
         "us_per_layer": 1e3 * ms_per_step,
         "us_per_layer_p50": 1e3 * statistics.median(step_ms),
         "us_per_layer_direct_launch": 1e3 * direct_ms,
@@ -462,6 +472,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch-invariant", action="store_true",
+                    help="time moe_forward_batch_invariant (bf16 workloads)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="override T of the workload (smaller cases for profiler captures)")
     ap.add_argument("--experts", type=int, default=None,

@@ -118,6 +118,27 @@ moe_status_t moe_forward(const void *hidden, const void *router_w, const float *
                          void *out, void *workspace, size_t workspace_bytes,
                          moe_debug_out_t *dbg, void *stream);
 
+/* Batch-invariant form of moe_forward (bf16 only): the output row of a
+ * token is bit-identical whatever other tokens share the call and whatever
+ * its position in the batch.  (The pages' second theme is bit-exact
+ * inference across processes for RL, "Fused MoE on Hopper, bit-exact vLLM
+ * across processes, and linear attention on TPUs", TL;DR and key points;
+ * this mode gives the layer that property with respect to batching.)  Every
+ * element is produced by the same sequence of operations for any T: one
+ * logits kernel with a fixed summation order (no split over H), exact
+ * routing, the swap-AB orientation for every expert with the MMA's token
+ * dimension fixed at 64, whole tiles per CTA (no split of the reduction
+ * dimension across CTAs), and the slot-ordered combine.  Same arguments,
+ * workspace (bf16) and errors as moe_forward, without the dtype and FP8
+ * scale arguments: per-tensor FP8 scales depend on the whole batch, so this
+ * mode is bf16 only.  Slower than moe_forward for large T (no normal
+ * orientation, no split of the reduction across CTAs). */
+moe_status_t moe_forward_batch_invariant(const void *hidden, const void *router_w,
+                                         const float *router_bias, const void *w13, const void *w2,
+                                         int T, int H, int E, int I, int top_k, void *out,
+                                         void *workspace, size_t workspace_bytes,
+                                         moe_debug_out_t *dbg, void *stream);
+
 /* moe_forward with host-side activations: copies hidden_host [T, H] bf16
  * (pinned host memory) into the workspace, runs the layer, and copies the
  * result into out_host [T, H] bf16 (pinned host memory), all enqueued on

@@ -23,7 +23,8 @@ STATUS = {
 
 # every symbol include/moe.h declares
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_forward", "moe_forward_hostio",
-           "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static")
+           "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static",
+           "moe_forward_batch_invariant")
 
 
 class DebugOut(C.Structure):
@@ -59,6 +60,8 @@ def lib() -> C.CDLL:
         L.moe_workspace_init.argtypes = [vp, sz, vp]
         L.moe_forward.restype = i
         L.moe_forward.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, C.POINTER(DebugOut), vp]
+        L.moe_forward_batch_invariant.restype = i
+        L.moe_forward_batch_invariant.argtypes = [vp] * 5 + [i] * 5 + [vp, vp, sz, vp, vp]
         L.moe_forward_hostio.restype = i
         L.moe_forward_hostio.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, vp]
         L.moe_route.restype = i

@@ -157,9 +157,10 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                           const void* w13, const void* w2, const float* w13_scale,
                           const float* w2_scale, int T, int H, int E, int I, int k, int dtype,
                           void* out, void* ws, size_t ws_bytes, moe_debug_out_t* dbg,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool invariant = false) {
   MOE_TRY(check_shape(T, H, E, I, k, dtype));
   const bool fp8 = dtype == MOE_DTYPE_FP8_E4M3;
+  if (invariant && fp8) return MOE_ERR_INVALID_ARG;   // per-tensor FP8 scales span the batch
   if (!hidden || !router_w || !w13 || !w2 || !out || !ws) return MOE_ERR_INVALID_ARG;
   if (fp8 && (!w13_scale || !w2_scale)) return MOE_ERR_INVALID_ARG;
   if (!aligned16(hidden) || !aligned16(router_w) || !aligned16(w13) || !aligned16(w2) ||
@@ -174,6 +175,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   if (dbg && dbg->force_orient == 1) tau = INT_MAX;
   if (dbg && dbg->force_orient == 2) tau = 0;
   if (H % 256 != 0) tau = INT_MAX;   // the normal-orientation w2 tile is 256 rows of H
+  if (invariant) tau = INT_MAX;       // one orientation for every expert and batch
   const bool any_swap = tau > 0;
   const bool any_normal = T > tau;
 
@@ -201,7 +203,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 router_bias, T, H, E, k,
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
-                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit)};
+                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0};
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
@@ -237,6 +239,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                        ? static_cast<unsigned long long>(dbg->wait_timeout_us) * 1000ull
                        : kWaitTimeoutNs;
   g13.inject_stall = dbg ? dbg->inject_stall : 0;
+  g13.whole_units = invariant ? 1 : 0;
   float* amax_cta = at<float>(ws, L.amax_cta);
   if (any_swap) {
     GemmArgs g = g13;
@@ -338,6 +341,16 @@ moe_status_t moe_forward(const void* hidden, const void* router_w, const float* 
   return forward_impl(hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I,
                       top_k, dtype, out, workspace, workspace_bytes, dbg,
                       static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_batch_invariant(const void* hidden, const void* router_w,
+                                         const float* router_bias, const void* w13, const void* w2,
+                                         int T, int H, int E, int I, int top_k, void* out,
+                                         void* workspace, size_t workspace_bytes,
+                                         moe_debug_out_t* dbg, void* stream) {
+  return forward_impl(hidden, router_w, router_bias, w13, w2, nullptr, nullptr, T, H, E, I, top_k,
+                      MOE_DTYPE_BF16, out, workspace, workspace_bytes, dbg,
+                      static_cast<cudaStream_t>(stream), true);
 }
 
 moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,

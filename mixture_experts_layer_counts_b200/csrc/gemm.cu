@@ -257,14 +257,20 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
   const long long W = nunits * ksteps;
   // Swap-AB: contiguous balanced atom ranges (units may be split across CTAs).
   // Normal orientation: whole units dealt round-robin in the grouped order.
-  constexpr bool kRR = !C::kSwap;
+  constexpr bool kRR = !C::kSwap;   // grouped unit order (normal orientation)
+  const bool rr = kRR || a.whole_units != 0;
+  // swap-AB token columns of a chunk of nv tokens: rounded up to 16, or the
+  // largest chunk when every element must see the same MMA shape
+  auto swap_cols = [&](int nv) {
+    return a.whole_units ? C::kBN : (nv + kTokenBox - 1) / kTokenBox * kTokenBox;
+  };
   int G = static_cast<int>(W / kMinAtomsPerCta);
   G = G < 1 ? 1 : (G > static_cast<int>(gridDim.x) ? static_cast<int>(gridDim.x) : G);
-  const bool active = kRR ? static_cast<long long>(blockIdx.x) < nunits
+  const bool active = rr ? static_cast<long long>(blockIdx.x) < nunits
                           : (W > 0 && static_cast<int>(blockIdx.x) < G);
-  const long long my_a0 = (active && !kRR) ? range_begin(W, G, blockIdx.x) : 0;
-  const long long my_a1 = (active && !kRR) ? range_begin(W, G, blockIdx.x + 1) : 0;
-  const Segments seg0{my_a0, my_a1, ksteps, kRR, static_cast<long long>(blockIdx.x), nunits,
+  const long long my_a0 = (active && !rr) ? range_begin(W, G, blockIdx.x) : 0;
+  const long long my_a1 = (active && !rr) ? range_begin(W, G, blockIdx.x + 1) : 0;
+  const Segments seg0{my_a0, my_a1, ksteps, rr, static_cast<long long>(blockIdx.x), nunits,
                       static_cast<int>(gridDim.x)};
 
   const bool producer = warp == 0 && lane == 0 && active;
@@ -287,7 +293,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const int wrow0 = e * a.w_rows_per_expert + mt * (C::kSwap ? kTileM : C::kBN);
-      const int nbox = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox : 0;
+      const int nbox = C::kSwap ? swap_cols(nv) / kTokenBox : 0;
       if (a.inject_stall != 0 && blockIdx.x == 0 && first) return;
       uint8_t* st = tiles + stage * C::kStageBytes;
 #pragma unroll
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
         int4 ch;
         int mt;
         unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
-        const int nvpad = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
+        const int nvpad = swap_cols(ch.z);
         return KA * (C::kNumA * C::kATile + nvpad * kAtomBytes);
       } else if constexpr (C::kPair) {
         int4 ch;
@@ -411,7 +417,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       int n;
       if constexpr (C::kSwap) {
-        n = (ch.z + kTokenBox - 1) / kTokenBox * kTokenBox;
+        n = swap_cols(ch.z);
       } else {
         n = C::kNumAcc * C::kBN;   // 256: w13 gate + up in one MMA, w2 one tile
       }
@@ -480,9 +486,9 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       unit_coords<kRR, C::kChunkTokens>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y, nv = ch.z;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
-      const int ncols = C::kSwap ? (nv + kTokenBox - 1) / kTokenBox * kTokenBox : C::kBN;
+      const int ncols = C::kSwap ? swap_cols(nv) : C::kBN;
 
-      if (!kRR && kb0 > 0) {   // (whole units only in the round-robin schedule)
+      if (!rr && kb0 > 0) {   // (whole units only in the round-robin schedule)
         // ---- later piece of a split unit: hand the raw accumulator over ----
         float* slot = a.partials + static_cast<size_t>(blockIdx.x) * kPartialSlotFloats;
         for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -509,7 +515,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
 
       // ---- first atoms of the unit: collect the later pieces, then finish ----
       int last = blockIdx.x;
-      if (!kRR && kb1 < ksteps) {
+      if (!rr && kb1 < ksteps) {
         const long long unit_end = (static_cast<long long>(u) + 1) * ksteps;
         last = atom_owner(unit_end - 1, W, G);
         bool ok = true;

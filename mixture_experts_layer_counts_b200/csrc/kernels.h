@@ -58,6 +58,7 @@ struct RouterArgs {
   unsigned char* cand;
   uint32_t* hdr;
   float* rsplit;          // router_split_floats(T, E) floats, or NULL (no split-K)
+  int invariant;          // 1: one logits kernel and summation order for every T (no split-K)
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 
@@ -114,6 +115,9 @@ struct GemmArgs {
   int* flags;                  // kMaxSlots flags, zero at launch
   unsigned long long timeout_ns;   // limit of every bounded wait in the kernel
   int inject_stall;            // failure-path test: CTA 0 leaves one stage unfilled
+  int whole_units;             // 1: whole units dealt round-robin (no K splits) and, for
+                               // swap-AB, MMA N fixed at the largest chunk: every output
+                               // element then sees the same operations whatever the batch
 };
 
 enum class Orient { kSwap, kNormal };

@@ -763,6 +763,78 @@ static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, in
                     a.T, a.H, a.E, a.k, gamma, ulast, a.topk_ids, a.topk_w, a.cand, a.hdr);
 }
 
+// ---------------------------------------------------------------------------
+// Kernel 1c (batch-invariant calls with small batches): the tiled kernel's
+// exact arithmetic (unsplit) at one token per CTA, one expert per warp.  Lane
+// l forms the fp32 FMA chains of K tiles l, l + 32, ... (64 products each, in
+// K order, from zero); lane 0 then adds the tile sums in K-tile order from
+// zero and adds the bias, so every logit is bit-identical to the tiled
+// kernel's for any batch size.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) router_logits_blocked_kernel(
+    const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
+    const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok) {
+  pdl_wait();
+  pdl_launch_next();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int e = blockIdx.y * 8 + warp;
+  const int vpr = H / 8;
+  const int ntiles = H / kLgK;            // 64-element K tiles
+  const uint4* xv = reinterpret_cast<const uint4*>(hidden) + static_cast<size_t>(t) * vpr;
+  if (blockIdx.y == 0 && warp == 0) {     // ||x_t|| and amax|x_t| (certification, FP8 scale)
+    float ss = 0.f, am = 0.f;
+    for (int c = lane; c < vpr; c += 32) {
+      float f[8];
+      unpack8(xv[c], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ss = fmaf(f[i], f[i], ss);
+        am = fmaxf(am, fabsf(f[i]));
+      }
+    }
+    ss = warp_sum(ss);
+    am = warp_max(am);
+    if (lane == 0) {
+      xnorm[t] = sqrtf(ss);
+      amax_tok[t] = am;
+    }
+  }
+  if (e >= E) return;
+  const uint4* wv = reinterpret_cast<const uint4*>(router_w) + static_cast<size_t>(e) * vpr;
+  float acc = 0.f, wsq = 0.f;
+  for (int j0 = 0; j0 < ntiles; j0 += 32) {
+    const int j = j0 + lane;
+    float tsum = 0.f;
+    if (j < ntiles) {
+#pragma unroll
+      for (int q = 0; q < kLgK / 8; ++q) {
+        float xf[8], wf[8];
+        unpack8(xv[j * (kLgK / 8) + q], xf);
+        unpack8(wv[j * (kLgK / 8) + q], wf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          tsum = fmaf(xf[i], wf[i], tsum);
+          wsq = fmaf(wf[i], wf[i], wsq);
+        }
+      }
+    }
+    // tile sums added in K-tile order by lane 0
+    const int nj = min(32, ntiles - j0);
+    for (int i = 0; i < nj; ++i) {
+      const float v = __shfl_sync(0xffffffffu, tsum, i);
+      if (lane == 0) acc += v;
+    }
+  }
+  wsq = warp_sum(wsq);
+  if (lane == 0) {
+    const float b = bias ? bias[e] : 0.f;
+    logits[static_cast<size_t>(t) * E + e] = acc + b;
+    if (t == 0) wnorm[e] = sqrtf(wsq);
+  }
+}
+
 static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStream_t st) {
   auto kern = router_logits_tiled_kernel;
   const int smem = 2 * (kLgT + kLgE) * kLgLd * 4;
@@ -781,21 +853,28 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   // fp32 with the wider certified bound for large batches
   const double macs = static_cast<double>(a.T) * a.E * a.H;
   const bool acc64 = macs <= static_cast<double>(1 << 28);
-  const int mode = !acc64 ? kAcc32 : (macs <= static_cast<double>(1 << 25) ? kAcc64 : kAccMixed);
+  int mode = !acc64 ? kAcc32 : (macs <= static_cast<double>(1 << 25) ? kAcc64 : kAccMixed);
   cudaError_t err;
   int nchain;
   int nsplit = 1;
-  if (!acc64 && a.E >= 32) {
+  if (a.invariant || (!acc64 && a.E >= 32)) {
     // large batch: register-tiled fp32 GEMM (blocked summation, see above),
     // split over K until the grid fills two CTAs per SM
     const int tiles = ((a.T + kLgT - 1) / kLgT) * ((a.E + kLgE - 1) / kLgE);
-    if (a.rsplit != nullptr) {
+    if (a.rsplit != nullptr && !a.invariant) {
       const int want = (2 * current_sm_count() + tiles - 1) / tiles;
       nsplit = want < 1 ? 1 : (want > kRouterSplits ? kRouterSplits : want);
       if (nsplit > a.H / kLgK) nsplit = a.H / kLgK;
     }
-    err = launch_logits_tiled(a, nsplit, st);
+    const bool blocked = a.invariant && tiles < current_sm_count();
+    if (blocked)   // the same arithmetic, spread over more SMs
+      err = launch_pdl(router_logits_blocked_kernel, dim3(a.T, (a.E + 7) / 8), dim3(256), 0, st,
+                       a.hidden, a.router_w, a.bias, a.T, a.H, a.E, a.logits, a.xnorm, a.wnorm,
+                       a.amax_tok);
+    else
+      err = launch_logits_tiled(a, nsplit, st);
     nchain = a.H / kLgK + 64;
+    mode = kAcc32;
   } else {
     // tokens per CTA: the largest of 16, 8, 4, 2 that still gives two waves
     // of CTAs (fewer tokens per CTA means more re-reads of router rows from
@@ -837,7 +916,7 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
   const float gamma = mode == kAcc64     ? static_cast<float>(nchain * u64 * 1.0001)
                       : mode == kAccMixed ? static_cast<float>((7.0 * u32 + nchain * u64) * 1.0001)
                                           : static_cast<float>(nchain * u32 * 1.0001);
-  const float ulast = acc64 ? static_cast<float>(u32) : static_cast<float>(2.0 * u32);
+  const float ulast = mode != kAcc32 ? static_cast<float>(u32) : static_cast<float>(2.0 * u32);
   if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, nsplit, st);
   if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, nsplit, st);
   return launch_topk<kMaxExperts / 32>(a, gamma, ulast, nsplit, st);

@@ -61,13 +61,15 @@ def make_workspace(T, H, E, I, top_k, dtype, device="cuda") -> torch.Tensor:
 def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w2_scale=None,
                 out=None, workspace=None, debug: dict | None = None, stream=None,
                 force_orient: int = 0, stage_events=None, wait_timeout_us: int = 0,
-                inject_stall: int = 0) -> torch.Tensor:
+                inject_stall: int = 0, batch_invariant: bool = False) -> torch.Tensor:
     """out[T, H] bf16 of the fused MoE layer (see include/moe.h).
 
     ``debug``: optional dict; keys filled on return (device tensors):
     topk_ids, topk_w, counts, offsets, perm, inv_perm, inter, act_scales.
     ``stage_events``: optional list of 8 torch.cuda.Event recorded at the
     stage boundaries on the launch stream.
+    ``batch_invariant``: call moe_forward_batch_invariant (bf16 only): each
+    token's output row is independent of the rest of the batch.
     """
     _need(hidden, torch.bfloat16, "hidden")
     _need(router_w, torch.bfloat16, "router_w")
@@ -111,6 +113,14 @@ def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w
             dbg.stage_events = C.cast(arr, C.c_void_p)
         dbg_p = C.pointer(dbg)
         keep.append(dbg)
+    if batch_invariant:
+        if dt != MOE_DTYPE_BF16 or w13_scale is not None or w2_scale is not None:
+            raise TypeError("the batch-invariant layer is bf16 only")
+        rc = _lib.lib().moe_forward_batch_invariant(
+            _ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(w13), _ptr(w2), T, H, E, I, top_k,
+            _ptr(out), _ptr(workspace), workspace.numel(), dbg_p, _stream(stream))
+        check(rc, "moe_forward_batch_invariant")
+        return out
     rc = _lib.lib().moe_forward(
         _ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(w13), _ptr(w2), _ptr(w13_scale),
         _ptr(w2_scale), T, H, E, I, top_k, dt, _ptr(out), _ptr(workspace), workspace.numel(),
