@@ -69,10 +69,20 @@ def kernel_traffic(workload):
     d = json.load(open(p)).get(workload)
     if not d:
         return None
-    src = open(os.path.join(ROOT, "mixture_experts_layer_counts_b200", "csrc", "gemm.cu"), "rb").read()
-    if hashlib.sha256(src).hexdigest()[:16] != d.get("gemm_cu_sha"):
+    if code_sha(os.path.join(ROOT, "mixture_experts_layer_counts_b200", "csrc", "gemm.cu")) != d.get("gemm_cu_sha"):
         return None
     return d.get("dram_bytes_per_launch")
+
+
+def code_sha(path):
+    """Hash of a C++ source without its // comments and blank lines (a
+    comment edit leaves the captured counters valid; a code edit does not)."""
+    lines = []
+    for ln in open(path, encoding="utf-8"):
+        code = ln.split("//", 1)[0].strip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
 class ClockSampler:

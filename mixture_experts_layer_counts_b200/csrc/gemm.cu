@@ -10,39 +10,53 @@
 //             tokens, D[weight row, token] in TMEM.  Used for experts with few
 //             tokens: every weight byte is streamed once, the MMA N is the
 //             token count rounded up to 16.
-//   kNormal : A (M = 128) = 128 tokens of one expert, B (N = 128 or 256) =
-//             weight rows, D[token, weight row].  Used for experts with many
-//             tokens (prefill-sized batches), where the MMA tile is full.
+//   kNormal : A (M = 128) = 128 tokens of one expert, B (N = 256) = weight
+//             rows, D[token, weight row].  Used for experts with many tokens
+//             (prefill-sized batches), where the MMA tile is full.  The
+//             gate/up GEMM stages two 128-token M tiles (a 256-token chunk)
+//             per weight tile, so each staged weight byte feeds two MMAs.
 // Projections.
-//   kW13 : two accumulators per tile, gate rows [i, i+.) and up rows
-//          [I+i, I+i+.) of w13[e], so one thread holds g and u of the same
-//          (token, i) and the epilogue forms h = SiLU(g) * u directly:
+//   kW13 : gate rows [i, i+.) and up rows [I+i, I+i+.) of w13[e] in two
+//          accumulators (swap-AB: two MMAs; normal: one N = 256 MMA over the
+//          adjacent gate and up tiles), so one thread holds g and u of the
+//          same (token, i) and the epilogue forms h = SiLU(g) * u directly:
 //          bf16 path -> inter (bf16, RNE); FP8 path -> h (fp32) + per-CTA
 //          amax|h| for the per-tensor requantisation that follows.
 //   kW2  : one accumulator; the epilogue multiplies by the router weight
 //          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), which
 //          the combine pass sums in slot order: deterministic, no atomics.
 //
-// Work split (balanced over the persistent CTAs).  A "unit" is one output
-// tile (token chunk x weight-row tile) and needs `katoms` K atoms.  The
-// nunits * katoms atoms are cut into G equal contiguous ranges, one per CTA,
-// so every SM streams the same number of weight bytes whatever the number of
-// active experts.  A unit cut by a range boundary is finished by the CTA that
-// holds its first atoms (the "head", whose range ends there, so it reaches
-// that unit last): the CTAs holding the later atoms write their fp32 partial
-// accumulators to their own slot and raise a flag; the head adds the partials
-// in K order and runs the epilogue.  Fixed order, no atomics on data.
+// Work split.  A "unit" is one output tile (token chunk x weight-row tile)
+// and needs `katoms` K atoms.
+//   Swap-AB (HBM-bound): the nunits * katoms atoms are cut into G equal
+//   contiguous ranges, one per CTA, so every SM streams the same number of
+//   weight bytes whatever the number of active experts.  A unit cut by a
+//   range boundary is finished by the CTA that holds its first atoms (the
+//   "head", whose range ends there, so it reaches that unit last): the CTAs
+//   holding the later atoms write their fp32 partial accumulators to their
+//   own slot and raise a flag; the head adds the partials in K order and runs
+//   the epilogue.  Fixed order, no atomics on data.
+//   Normal (tensor-bound), and swap-AB in the batch-invariant mode: whole
+//   units dealt round-robin; normal units ordered expert -> weight tile ->
+//   token chunk, so the chunks sharing a weight tile run on neighbouring SMs
+//   at the same time and the tile is read from DRAM about once.
 //
-// Pipeline per CTA (192 threads):
+// Pipeline per CTA:
 //   warp 0 lane 0  TMA producer: STAGES-deep ring of {A, B} tiles, 128-byte
 //                  K atoms in the 128B-swizzle layout, mbarrier complete_tx.
+//                  The tile schedule is complete when the kernel starts, so
+//                  the first stages' weight tiles are requested before the
+//                  wait for the previous kernel's activations.
 //   warp 1 lane 0  MMA issuer: 4 MMAs (K = 16 bf16 / 32 E4M3 each) per atom
 //                  and accumulator; tcgen05.commit frees the smem slot; a
 //                  final commit hands the TMEM buffer to the epilogue.
-//   warps 2..5     epilogue: tcgen05.ld 32 lanes x 16 columns per warp
-//                  (warp w reads TMEM lanes 32*(w%4)..+31), math, stores.
-// Two TMEM accumulator buffers, so the epilogue of one segment overlaps the
-// mainloop of the next.  Every wait is bounded (see mbar_wait).
+//   warps 2..      epilogue (4 warps for swap-AB, 8 for normal: two per TMEM
+//                  lane quadrant, warp w reads lanes 32*(w%4)..+31):
+//                  tcgen05.ld, math, stores (normal: staged through smem so
+//                  whole row segments are written).
+// TMEM: two accumulator buffers (the epilogue of one unit overlaps the
+// mainloop of the next), except the 256-token gate/up units, whose two M
+// tiles fill all 512 columns.  Every wait is bounded (see mbar_wait).
 #include <cuda.h>
 #include <cuda_bf16.h>
 
