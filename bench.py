@@ -216,6 +216,16 @@ def blas_threads():
         return os.cpu_count()
 
 
+def cpu_model():
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def run_reference(args, wl, rank, world):
     if rank != 0:
         return
@@ -236,7 +246,8 @@ def run_reference(args, wl, rank, world):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": f"{args.workload}: {describe(wl)}", "sample": f"{len(toks)} of {wl['T']} tokens"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu": cpu_model(),
+                         "kind": "oracle",
                          "sample": f"fp64 oracle, tokens 0..{len(toks) - 1} of the {args.workload} batch "
                                    f"(full routing of all {wl['T']} tokens) per step"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -409,6 +420,12 @@ def run_ours(args, wl, rank, world, local):
     e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world)
     e2e_value = world * T * e2e_steps / (e2e_ms * 1e-3)
 
+    # every algorithmic byte of the call: activated weights once, router
+    # weights, hidden in, out, and the intermediates written and read once
+    # (x in perm order, the intermediate h, the fp32 weighted slot rows)
+    ab = esize
+    all_bytes = (weight_bytes + E * H * 2 + T * H * 2 + T * H * 2 + 2 * T * k * H * ab +
+                 2 * T * k * I * ab + 2 * T * k * H * 4)
     peak, peak_tf, peak_kind = peaks()
     w13_s = w13_kernel_ms * 1e-3
     # The w13 GEMM bracket is the dominant kernel.  Decode batches (a few
@@ -455,6 +472,8 @@ def run_ours(args, wl, rank, world, local):
         "weight_gbs_frac_of_measured_hbm": weight_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
         "weight_gbs_frac_of_8tbs": weight_bytes / (ms_per_step * 1e-3) / 8e12,
         "layer_tflops": 2.0 * T * k * 3 * I * H / (ms_per_step * 1e-3) / 1e12,
+        "all_bytes": all_bytes,
+        "all_gbs": all_bytes / (ms_per_step * 1e-3) / 1e9,
         "stages_us": {k_: 1e3 * v for k_, v in stage_ms.items()},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
@@ -467,6 +486,7 @@ def run_ours(args, wl, rank, world, local):
         toks = list(range(min(CPU_BASELINE_TOKENS, T)))
         secs = oracle_sample_seconds(host, wl, toks)
         line["cpu_baseline"] = {"value": len(toks) / secs, "unit": "tokens/s", "cores": blas_threads(),
+                                "cpu": cpu_model(),
                                 "kind": "oracle",
                                 "sample": f"fp64 oracle on tokens 0..{len(toks) - 1} of the batch "
                                           f"(routing of all {T} tokens), {secs:.1f} s"}
