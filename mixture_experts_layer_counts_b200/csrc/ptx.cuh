@@ -3,7 +3,8 @@
 //
 // Encodings follow the PTX ISA (tcgen05 "Matrix descriptors" and "Instruction
 // descriptor" tables).  Only the forms used by this library are wrapped.
-// No load here uses .multicast::cluster.
+// Every TMA load here fills only the issuing CTA's shared memory (no
+// cluster-wide delivery).
 #pragma once
 #include <cstdint>
 
