@@ -7,8 +7,7 @@ from oracle import bf16_tolerance_violation, moe_forward_ref, rel_l2
 
 # Router weights are fp32 softmax values renormalised over the top k, from
 # fp32 logits whose error is bounded by the router's certified bound; the
-# induced weight error stays below this (observed: about 1e-7 at decode
-# sizes, a few 1e-6 at the largest test shapes).
+# induced weight error stays below this.
 WEIGHT_ATOL = 2e-5
 
 
