@@ -315,6 +315,105 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   return MOE_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Launch cache.  A layer call enqueues about ten kernels; a caller that
+// repeats a call with identical arguments (a decode loop) gets it replayed
+// from an instantiated CUDA graph, one host launch instead of ten.  The first
+// call with a key runs directly (and performs every one-time initialisation);
+// the second records the same enqueue sequence on an internal stream that is
+// only ever captured, instantiates the graph and launches it on the caller's
+// stream; later calls launch the cached graph.  Calls made while the caller's
+// stream is being captured, and calls with debug outputs, run directly.  A
+// graph reads its buffers at replay time, so new contents at the same
+// addresses are seen; any change of pointer or size is a different key.
+struct CallKey {
+  int kind;
+  int dev;
+  const void* p[9];
+  long long n[7];
+  bool operator==(const CallKey& o) const {
+    if (kind != o.kind || dev != o.dev) return false;
+    for (int i = 0; i < 9; ++i)
+      if (p[i] != o.p[i]) return false;
+    for (int i = 0; i < 7; ++i)
+      if (n[i] != o.n[i]) return false;
+    return true;
+  }
+};
+
+struct CacheEntry {
+  CallKey key;
+  int state;               // 0 empty, 1 seen once, 2 graph ready, 3 capture failed
+  cudaGraphExec_t exec;
+  unsigned long long used;
+};
+
+constexpr int kCacheEntries = 32;
+
+template <class Enqueue>
+moe_status_t run_cached(const CallKey& key, cudaStream_t st, Enqueue&& enqueue) {
+  static std::mutex mu;
+  static CacheEntry cache[kCacheEntries];
+  static cudaStream_t capture_stream[kMaxDevices] = {};
+  static unsigned long long clock = 0;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+    return enqueue(st);
+  std::lock_guard<std::mutex> lock(mu);
+  CacheEntry* e = nullptr;
+  for (int i = 0; i < kCacheEntries; ++i)
+    if (cache[i].state != 0 && cache[i].key == key) e = &cache[i];
+  if (e == nullptr) {   // first sighting: remember the key, run directly
+    CacheEntry* v = &cache[0];
+    for (int i = 0; i < kCacheEntries; ++i) {
+      if (cache[i].state == 0) {
+        v = &cache[i];
+        break;
+      }
+      if (cache[i].used < v->used) v = &cache[i];
+    }
+    if (v->state == 2) cudaGraphExecDestroy(v->exec);
+    *v = CacheEntry{key, 1, nullptr, ++clock};
+    return enqueue(st);
+  }
+  e->used = ++clock;
+  if (e->state == 3) return enqueue(st);
+  if (e->state == 1) {
+    if (key.dev < 0 || key.dev >= kMaxDevices) {
+      e->state = 3;
+      return enqueue(st);
+    }
+    if (capture_stream[key.dev] == nullptr &&
+        cudaStreamCreateWithFlags(&capture_stream[key.dev], cudaStreamNonBlocking) != cudaSuccess) {
+      capture_stream[key.dev] = nullptr;
+      e->state = 3;
+      return enqueue(st);
+    }
+    cudaStream_t cap = capture_stream[key.dev];
+    cudaGraph_t graph = nullptr;
+    bool ok = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    if (ok) {
+      const moe_status_t rc = enqueue(cap);
+      const cudaError_t end = cudaStreamEndCapture(cap, &graph);
+      ok = rc == MOE_OK && end == cudaSuccess && graph != nullptr;
+      if (ok) ok = cudaGraphInstantiate(&e->exec, graph, 0ULL) == cudaSuccess;
+      if (graph != nullptr) cudaGraphDestroy(graph);
+    }
+    cudaGetLastError();   // a failed capture leaves no sticky error
+    if (!ok) {
+      e->state = 3;
+      return enqueue(st);
+    }
+    e->state = 2;
+  }
+  return cuda_status(cudaGraphLaunch(e->exec, st));
+}
+
+int current_device() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess ? dev : -1;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -338,9 +437,16 @@ moe_status_t moe_forward(const void* hidden, const void* router_w, const float* 
                          const float* w2_scale, int T, int H, int E, int I, int top_k, int dtype,
                          void* out, void* workspace, size_t workspace_bytes, moe_debug_out_t* dbg,
                          void* stream) {
-  return forward_impl(hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I,
-                      top_k, dtype, out, workspace, workspace_bytes, dbg,
-                      static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto enqueue = [&](cudaStream_t s) {
+    return forward_impl(hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I,
+                        top_k, dtype, out, workspace, workspace_bytes, dbg, s);
+  };
+  if (dbg != nullptr || check_shape(T, H, E, I, top_k, dtype) != MOE_OK) return enqueue(st);
+  const CallKey key{0, current_device(),
+                    {hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, out, workspace},
+                    {T, H, E, I, top_k, dtype, static_cast<long long>(workspace_bytes)}};
+  return run_cached(key, st, enqueue);
 }
 
 moe_status_t moe_forward_batch_invariant(const void* hidden, const void* router_w,
@@ -348,9 +454,16 @@ moe_status_t moe_forward_batch_invariant(const void* hidden, const void* router_
                                          int T, int H, int E, int I, int top_k, void* out,
                                          void* workspace, size_t workspace_bytes,
                                          moe_debug_out_t* dbg, void* stream) {
-  return forward_impl(hidden, router_w, router_bias, w13, w2, nullptr, nullptr, T, H, E, I, top_k,
-                      MOE_DTYPE_BF16, out, workspace, workspace_bytes, dbg,
-                      static_cast<cudaStream_t>(stream), true);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto enqueue = [&](cudaStream_t s) {
+    return forward_impl(hidden, router_w, router_bias, w13, w2, nullptr, nullptr, T, H, E, I,
+                        top_k, MOE_DTYPE_BF16, out, workspace, workspace_bytes, dbg, s, true);
+  };
+  if (dbg != nullptr || check_shape(T, H, E, I, top_k, MOE_DTYPE_BF16) != MOE_OK) return enqueue(st);
+  const CallKey key{1, current_device(),
+                    {hidden, router_w, router_bias, w13, w2, nullptr, nullptr, out, workspace},
+                    {T, H, E, I, top_k, MOE_DTYPE_BF16, static_cast<long long>(workspace_bytes)}};
+  return run_cached(key, st, enqueue);
 }
 
 moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
@@ -366,10 +479,16 @@ moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
   void* din = at<void>(workspace, L.staging_in);
   void* dout = at<void>(workspace, L.staging_out);
   const size_t bytes = static_cast<size_t>(T) * H * 2;
-  MOE_TRY(cuda_status(cudaMemcpyAsync(din, hidden_host, bytes, cudaMemcpyHostToDevice, st)));
-  MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
-                       dtype, dout, workspace, workspace_bytes, nullptr, st));
-  return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
+  auto enqueue = [&](cudaStream_t s) {
+    MOE_TRY(cuda_status(cudaMemcpyAsync(din, hidden_host, bytes, cudaMemcpyHostToDevice, s)));
+    MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
+                         dtype, dout, workspace, workspace_bytes, nullptr, s));
+    return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, s));
+  };
+  const CallKey key{2, current_device(),
+                    {hidden_host, router_w, router_bias, w13, w2, w13_scale, w2_scale, out_host, workspace},
+                    {T, H, E, I, top_k, dtype, static_cast<long long>(workspace_bytes)}};
+  return run_cached(key, st, enqueue);
 }
 
 moe_status_t moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,

@@ -283,3 +283,32 @@ def test_hostio_matches_device(cuda_ok):
     torch.cuda.synchronize()
     assert torch.equal(hout.view(torch.int16), ref.cpu().view(torch.int16))
     assert layer.get_status(ws)[0] == 0
+
+
+def test_repeated_calls_replay_a_graph_with_fresh_data(cuda_ok):
+    # identical arguments: run directly, then capture, then replay; every call
+    # must read the buffers' current contents
+    inp = custom_inputs(24, 512, 16, 256, 4, seed=21, bias=True)
+    T, H = inp["hidden"].shape
+    k = inp["top_k"]
+    ws = layer.make_workspace(T, H, inp["E"], inp["I"], k, 0)
+    out = torch.empty((T, H), dtype=torch.bfloat16, device="cuda")
+    hidden = inp["hidden"].clone()
+    hin = hidden.cpu().pin_memory()
+    hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
+    g = torch.Generator(device="cuda").manual_seed(5)
+    for it in range(4):
+        if it:
+            hidden.copy_(torch.randn(T, H, generator=g, device="cuda").to(torch.bfloat16))
+            hin.copy_(hidden.cpu())
+        ref = layer.moe_forward(hidden, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                                debug={})                    # debug outputs: always direct
+        layer.moe_forward(hidden, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                          out=out, workspace=ws)             # cached after the first call
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref)
+        layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
+                                 hout, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(hout.view(torch.int16), ref.cpu().view(torch.int16))
+    assert layer.get_status(ws)[0] == 0
