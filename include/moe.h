@@ -36,6 +36,12 @@
  *    enqueued.  Errors found on the device (a wait that timed out, an expert
  *    id out of range) are recorded in the workspace's status word and read
  *    with moe_get_status.
+ *  - Repeated calls of moe_forward / moe_forward_batch_invariant (without
+ *    debug outputs) or moe_forward_hostio with identical arguments are
+ *    replayed from a CUDA graph the library records on the second such call
+ *    (on an internal stream; nothing runs during the recording) and keeps
+ *    for up to 32 argument sets.  Buffers are read at replay time.  Calls on
+ *    a stream that is being captured always enqueue their kernels directly.
  *  - Shapes are runtime values; nothing is specialised per T (the pages'
  *    lesson about per-token-count JIT recompiles, "AWS details MoE kernel
  *    fixes...", third fix).  Results are deterministic: identical inputs give
