@@ -1,38 +1,48 @@
 """Benchmark of the fused MoE layer (one JSON line on rank 0).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode-fp8]
+                    [--impl ours|reference] [--only-headline]
 
 A step is one call of the whole layer (router, align, gather, w13 GEMM with
-SiLU*up, [FP8 requant], w2 GEMM with router-weighted slot scatter, combine)
-on one batch of synthetic decode tokens whose inputs already sit in HBM.
-Each rank runs its own batch (independent decode batches, weights replicated,
-no data-path collective): weak scaling, value = all ranks' tokens / the
-slowest rank's device time.  Between timed steps L2 is flushed by writing a
-256 MiB buffer; each step is timed alone with CUDA events on the launch
-stream, and the flush is outside the events.
+SiLU*up, [FP8 requantisation], w2 GEMM with router-weighted combine) on one
+batch of synthetic tokens whose inputs already sit in HBM.  The headline
+line times exactly K steps of the headline workload (default: decode-fp8,
+the largest decode layer: T=64 H=7168 E=256 top_k=8 I=2048, E4M3 W8A8);
+the key "workloads" carries the same fields for every one of the five layer
+shapes (tiny, decode, decode-zipf, decode-fp8, prefill-zipf), each timed
+over at least K steps and at least one second.  Each rank runs its own batch
+(independent batches, weights replicated, no data-path collective): weak
+scaling, value = all ranks' tokens / the slowest rank's device time.
+Between timed steps L2 is flushed by writing a 256 MiB buffer; each step is
+timed alone with CUDA events on the launch stream, and the flush is outside
+the events.
 
 Extra keys: us_per_layer, weight_bytes / weight_gbs (activated experts'
 weight bytes counted once per step), stages_us (per-kernel-stage device time
 from events the library records on the launch stream), roofline of the
-dominant kernel (w13 grouped GEMM, weight bytes of active experts / its
-measured time vs the measured HBM peak), e2e (same metric through the
-host-buffer C-ABI call with the H2D/D2H copies in the timed region),
-cpu_baseline (the fp64 oracle on a bounded token sample on the host cores),
-gpu_launches and clocks sampled with nvidia-smi during the timed region.
+dominant kernel (w13 grouped GEMM: weight bytes of the active experts / its
+time vs the measured HBM peak at decode; 2 T k 2I H flops / its time vs the
+measured bf16 peaks, burst and sustained, at prefill), e2e (same metric
+through the host-buffer C-ABI call with the H2D/D2H copies in the timed
+region), cpu_baseline (the fp64 oracle on a bounded token sample on the host
+cores), gpu_launches and SM clocks sampled through NVML during each timed
+region.
 
 --impl reference times the fp64 CPU oracle (the only other implementation of
-the layer; there is no installable reference package) on a bounded token
-sample per step, on rank 0 only.
+the layer; there is no installable reference package) on a bounded sample
+per step, on rank 0 only.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -44,21 +54,29 @@ import torch  # noqa: E402
 from mixture_experts_layer_counts_b200.inputs import WORKLOADS, describe, make_inputs  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
-REF_SAMPLE_TOKENS = 1          # tokens per --impl reference step
-CPU_BASELINE_TOKENS = 4        # tokens in the cpu_baseline sample
+HEADLINE = "decode-fp8"          # the largest decode layer
+ORDER = ["decode-fp8", "tiny", "decode", "decode-zipf", "prefill-zipf"]
+MIN_TIMED_S = 1.0                # each workload's timed region lasts at least this long
+REF_SAMPLE_TOKENS = 1            # tokens per --impl reference step
+CPU_BASELINE_TOKENS = 4          # tokens in the cpu_baseline sample
+# Fallbacks when MEASURED_PEAKS.json is absent: an earlier measurement of this
+# pool's B200s (HBM copy; cuBLAS bf16 GEMM burst and sustained under the power cap)
 FALLBACK_HBM_GBS = 6650.0
-
-
+FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0
 
 
 def peaks():
-    """(HBM GB/s, dense bf16 TFLOP/s sustained, kind): the driver's measured figures."""
+    """{hbm, bf16 burst, bf16 sustained, kind}: the measured figures of this
+    pool's B200s when MEASURED_PEAKS.json is present, else the fallbacks."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return float(d["hbm_gbs"]), float(d.get("bf16_tflops_sustained", d.get("bf16_tflops"))), "measured"
-    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
+        burst = float(d.get("bf16_tflops", d.get("bf16_tflops_sustained", FALLBACK_BF16_TFLOPS)))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=burst,
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", burst)), kind="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=FALLBACK_BF16_TFLOPS_SUSTAINED,
+                kind="fallback")
 
 
 def kernel_traffic(workload):
@@ -86,53 +104,64 @@ def code_sha(path):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """SM clock and clock-event reasons of this rank's GPU, sampled through NVML
+    every few milliseconds while the timed region runs (the GPU is found by
+    its PCI bus id, so the NVML index need not match the CUDA index)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, dev):
+    def __init__(self, dev, period_s=0.002):
         self.dev = dev
-        self.proc = None
+        self.period = period_s
+        self.sm, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def _handle(self):
+        import pynvml
+
+        pynvml.nvmlInit()
+        p = torch.cuda.get_device_properties(self.dev)
+        bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+
+    def _run(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        masks = [(n, getattr(nv, c, 0)) for n, c in self.REASONS]
+        while not self._stop.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                r = get_reasons(h)
+                for n, m in masks:
+                    if m and r & m:
+                        self.reasons.add(n)
+            except Exception:
+                pass
+            self._stop.wait(self.period)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            nv, h = self._handle()
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self._thread = threading.Thread(target=self._run, args=(nv, h), daemon=True)
+            self._thread.start()
+        except Exception:
+            self._thread = None
         return self
 
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        self._stop.set()
+        if self._thread:
+            self._thread.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 8:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.sm) if self.sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.sm)}
 
 
 def dist_setup(n_gpus):
@@ -185,13 +214,17 @@ def whole_job_tokens_per_s(world, T, steps, max_total_ms):
 
 
 def oracle_sample_seconds(inp_host, wl, tokens):
-    """Wall time of one oracle call on a token sample (inputs already on host)."""
+    """Wall time of one oracle call on a bounded sample of the batch (inputs
+    already on the host): the sampled tokens' rows form a layer call of their
+    own (routing, per-tensor scales and every expert product of those tokens).
+    The per-tensor FP8 scales then span the sample rather than the batch; the
+    work per token is the same."""
     from oracle import moe_forward_ref
 
+    hidden = inp_host["hidden"][list(tokens)]
     t0 = time.perf_counter()
-    moe_forward_ref(inp_host["hidden"], inp_host["router_w"], inp_host["bias"], inp_host["w13"],
-                    inp_host["w2"], wl["top_k"], wl["dtype"], inp_host["s13"], inp_host["s2"],
-                    tokens=tokens)
+    moe_forward_ref(hidden, inp_host["router_w"], inp_host["bias"], inp_host["w13"], inp_host["w2"],
+                    wl["top_k"], wl["dtype"], inp_host["s13"], inp_host["s2"])
     return time.perf_counter() - t0
 
 
@@ -233,23 +266,26 @@ def run_reference(args, wl, rank, world):
     inp = make_inputs(wl, dev, seed=wl["seed"])
     host = host_copy(inp)
     del inp
-    toks = list(range(REF_SAMPLE_TOKENS))
-    for _ in range(args.warmup):
-        oracle_sample_seconds(host, wl, toks)
-    times = [oracle_sample_seconds(host, wl, toks) for _ in range(args.steps)]
+    n_tok = min(REF_SAMPLE_TOKENS, wl["T"])
+    samples = [[(i * n_tok + j) % wl["T"] for j in range(n_tok)] for i in range(args.warmup + args.steps)]
+    for i in range(args.warmup):
+        oracle_sample_seconds(host, wl, samples[i])
+    times = [oracle_sample_seconds(host, wl, samples[args.warmup + i]) for i in range(args.steps)]
     total = sum(times)
-    value = len(toks) * args.steps / total
+    value = n_tok * args.steps / total
     cores = blas_threads()
     line = {
         "impl": "reference", "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus if hasattr(args, "gpus") else 1, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {describe(wl)}", "sample": f"{len(toks)} of {wl['T']} tokens"},
+        "config": {"workload": f"{args.workload}: {describe(wl)}",
+                   "sample": f"{n_tok} of {wl['T']} tokens per step"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "cpu": cpu_model(),
                          "kind": "oracle",
-                         "sample": f"fp64 oracle, tokens 0..{len(toks) - 1} of the {args.workload} batch "
-                                   f"(full routing of all {wl['T']} tokens) per step"},
+                         "sample": f"fp64 oracle; each step one token of the {args.workload} batch "
+                                   f"(tokens 0, 1, 2, ... in turn) as a one-token layer call: its routing, "
+                                   f"scales and its {wl['top_k']} experts' products"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -268,8 +304,39 @@ def launches_per_step(wl, T):
     return n + (1 if wl["dtype"] == "fp8" else 0)
 
 
-def run_ours(args, wl, rank, world, local):
+def new_events(n, stream):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for ev in evs:           # torch creates the CUDA event on first record
+        ev.record(stream)
+    return evs
+
+
+def time_graph_steps(graph, flush, stream, steps, world, local):
+    """Device time of `steps` replays of `graph`, each bracketed by events on
+    `stream`, with an L2 flush before each (outside the events).  Returns
+    (per-step ms list, max over ranks of the total ms, clock summary)."""
+    tev = [new_events(2, stream) for _ in range(steps)]
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(steps):
+            flush.zero_()
+            tev[i][0].record(stream)
+            graph.replay()
+            tev[i][1].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    step_ms = [a_.elapsed_time(b_) for a_, b_ in tev]
+    return step_ms, max_over_ranks(sum(step_ms), world), clk.summary()
+
+
+def measure_workload(name, wl, args, rank, world, local, steps_exact=None):
+    """Every figure of one workload (see the module docstring).  steps_exact:
+    time exactly that many steps; otherwise at least args.steps and at least
+    MIN_TIMED_S of device time."""
     from mixture_experts_layer_counts_b200 import layer
+    from mixture_experts_layer_counts_b200.layer import N_STAGE_EVENTS, STAGES
 
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
@@ -283,21 +350,20 @@ def run_ours(args, wl, rank, world, local):
     if args.batch_invariant:
         fwd["batch_invariant"] = True
 
-    def step(events=None):
+    def call(**kw):
         layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
-                          stage_events=events, **fwd)
+                          **fwd, **kw)
 
-    # warm-up (also yields the routing this batch produces)
+    # warm-up (the debug call also yields the routing this batch produces)
     dbg = {}
-    layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
-                      debug=dbg, **fwd)
+    call(debug=dbg)
     for _ in range(args.warmup):
         flush.zero_()
-        step()
+        call()
     torch.cuda.synchronize()
     code, info = layer.get_status(ws)
     if code != 0:
-        raise RuntimeError(f"device status {code} info {info:#x} after warm-up")
+        raise RuntimeError(f"{name}: device status {code} info {info:#x} after warm-up")
     counts = dbg["counts"].cpu().numpy()
     e_act = int((counts > 0).sum())
     esize = 1 if dt == 1 else 2
@@ -305,76 +371,60 @@ def run_ours(args, wl, rank, world, local):
     w2_bytes = e_act * H * I * esize
     weight_bytes = w13_bytes + w2_bytes
 
-    from mixture_experts_layer_counts_b200.layer import N_STAGE_EVENTS, STAGES
-
-    def new_events(n):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-        for ev in evs:           # torch creates the CUDA event on first record
-            ev.record(stream)
-        return evs
-
     # The timed step is one replay of a CUDA graph holding one layer call, the
-    # way a decode engine runs it (kernels chained by programmatic dependent
-    # launch).  Start/end events are recorded on the stream around each
-    # replay; the L2 flush sits between steps, outside the events.
+    # way an inference engine runs a layer (kernels chained by programmatic
+    # dependent launch).
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step()
+        call()
     for _ in range(3):
         flush.zero_()
         graph.replay()
-    tev = [new_events(2) for _ in range(args.steps)]
     torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(args.steps):
-            flush.zero_()
-            tev[i][0].record(stream)
-            graph.replay()
-            tev[i][1].record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
+    if steps_exact is not None:
+        steps = steps_exact
+    else:
+        probe, _, _ = time_graph_steps(graph, flush, stream, 5, 1, local)
+        per = max(statistics.median(probe), 1e-3) * 1e-3 + 40e-6     # + the flush
+        steps = max(args.steps, int(math.ceil(MIN_TIMED_S / per)))
+        steps = int(max_over_ranks(float(steps), world))
+    step_ms, total_ms, clocks = time_graph_steps(graph, flush, stream, steps, world, local)
     code, info = layer.get_status(ws)
     if code != 0:
-        raise RuntimeError(f"device status {code} info {info:#x} in the timed region")
-    step_ms = [a_.elapsed_time(b_) for a_, b_ in tev]
-    total_ms = max_over_ranks(sum(step_ms), world)
-    ms_per_step = total_ms / args.steps
-    value = whole_job_tokens_per_s(world, T, args.steps, total_ms)
+        raise RuntimeError(f"{name}: device status {code} info {info:#x} in the timed region")
+    ms_per_step = total_ms / steps
+    value = whole_job_tokens_per_s(world, T, steps, total_ms)
     del graph
 
-    # Per-kernel breakdown: the same graph with the library's 8 stage events
-    # recorded inside it (each event node costs ~2-3 us, so these stage times
-    # are upper bounds and their sum exceeds the step time above).
-    gev = new_events(N_STAGE_EVENTS)
+    # Per-kernel breakdown: the same graph with the library's stage events
+    # inside it (each event node costs ~2-3 us and breaks the programmatic
+    # launch overlap, so these stage times are upper bounds).
+    n_stage = min(steps, 300)
+    gev = new_events(N_STAGE_EVENTS, stream)
     torch.cuda.synchronize()
     igraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(igraph):
-        step(gev)
-    n_stage = min(args.steps, 1000)
+        call(stage_events=gev)
     stage_sum = [0.0] * (N_STAGE_EVENTS - 1)
     for i in range(n_stage + 3):
         flush.zero_()
         igraph.replay()
         gev[-1].synchronize()
         if i >= 3:
-            for s in range(1, N_STAGE_EVENTS):
-                stage_sum[s - 1] += gev[s - 1].elapsed_time(gev[s])
-    stage_ms = {STAGES[s]: stage_sum[s - 1] / n_stage for s in range(1, N_STAGE_EVENTS)}
+            for st in range(1, N_STAGE_EVENTS):
+                stage_sum[st - 1] += gev[st - 1].elapsed_time(gev[st])
+    stage_ms = {STAGES[st]: stage_sum[st - 1] / n_stage for st in range(1, N_STAGE_EVENTS)}
     del igraph
 
     # The dominant kernel alone: a graph whose only stage events bracket the
-    # w13 GEMM (entries 3 and 4), so the kernel is timed with one event node
-    # on each side instead of eight.
-    wev = new_events(2)
+    # w13 GEMM (entries 3 and 4).
+    wev = new_events(2, stream)
     sel = [None] * N_STAGE_EVENTS
     sel[3], sel[4] = wev[0], wev[1]
     torch.cuda.synchronize()
     wgraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(wgraph):
-        layer.moe_forward(inp["hidden"], inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
-                          stage_events=sel, **fwd)
+        call(stage_events=sel)
     w13_ms = []
     for i in range(n_stage + 3):
         flush.zero_()
@@ -386,19 +436,19 @@ def run_ours(args, wl, rank, world, local):
     w13_kernel_ms = statistics.mean(w13_ms)
 
     # the same step launched directly (no graph): host launch gaps included
-    n_direct = min(args.steps, 500)
-    dev_ = [new_events(N_STAGE_EVENTS) for _ in range(n_direct)]
+    n_direct = min(steps, 200)
+    dev_ = [new_events(N_STAGE_EVENTS, stream) for _ in range(n_direct)]
     torch.cuda.synchronize()
     for i in range(n_direct):
         flush.zero_()
-        step(dev_[i])
+        call(stage_events=dev_[i])
     torch.cuda.synchronize()
     direct_ms = max_over_ranks(sum(e[0].elapsed_time(e[-1]) for e in dev_), world) / n_direct
 
     # end to end: pinned host hidden in, pinned host out, copies inside the timed region
     hin = inp["hidden"].cpu().pin_memory()
     hout = torch.empty((T, H), dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(10, min(args.steps, 200))
+    e2e_steps = max(10, min(steps, 200))
     e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
     barrier(world)
     torch.cuda.synchronize()
@@ -408,8 +458,7 @@ def run_ours(args, wl, rank, world, local):
         e_ev[i][0].record(stream)
         if args.batch_invariant:   # no host-I/O entry point: the same copies around the call
             dev_hidden.copy_(hin, non_blocking=True)
-            layer.moe_forward(dev_hidden, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
-                              **fwd)
+            layer.moe_forward(dev_hidden, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k, **fwd)
             hout.copy_(out, non_blocking=True)
         else:
             layer.moe_forward_hostio(hin, inp["router_w"], inp["router_bias"], inp["w13"], inp["w2"], k,
@@ -426,70 +475,105 @@ def run_ours(args, wl, rank, world, local):
     ab = esize
     all_bytes = (weight_bytes + E * H * 2 + T * H * 2 + T * H * 2 + 2 * T * k * H * ab +
                  2 * T * k * I * ab + 2 * T * k * H * 4)
-    peak, peak_tf, peak_kind = peaks()
+    pk = peaks()
     w13_s = w13_kernel_ms * 1e-3
-    # The w13 GEMM bracket is the dominant kernel.  Decode batches (a few
-    # tokens per expert, swap-AB tiles) are bound by streaming the activated
-    # experts' weights: achieved = those bytes / time vs the measured HBM
-    # copy bandwidth.  Prefill batches (normal-orientation tiles) are bound by
-    # the tensor pipe: achieved = 2 * T*k * 2I * H / time vs the measured
-    # sustained bf16 GEMM rate (the kernel runs inside a long step).
-    tensor_bound = T * k / max(e_act, 1) > 64
+    flops = 2.0 * T * k * 3 * I * H
+    # The w13 GEMM is the dominant kernel.  Decode batches (a few tokens per
+    # expert, swap-AB tiles) are bound by streaming the activated experts'
+    # weights: achieved = those bytes / time vs the measured HBM copy
+    # bandwidth.  Prefill batches (normal-orientation tiles) are bound by the
+    # tensor pipe: achieved = 2 T k 2I H / time vs the measured bf16 GEMM rate,
+    # burst (the kernel timed on its own) and sustained (inside a long step).
+    tensor_bound = T * k / max(e_act, 1) > SWAP_MAX_TOKENS
     w13_flops = 2.0 * T * k * 2 * I * H
     if tensor_bound:
-        roof = {"kernel": "grouped_gemm_kernel<normal, w13>", "bound": "tensor",
-                "achieved": w13_flops / w13_s / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
-                "frac": w13_flops / w13_s / 1e12 / peak_tf, "peak_kind": peak_kind + " (bf16, sustained)",
+        mult = 2.0 if dt == 1 else 1.0      # E4M3: the nominal fp8 / bf16 ratio
+        ach = w13_flops / w13_s / 1e12
+        roof = {"kernel": "grouped_gemm_kernel<normal, w13>", "bound": "tensor", "achieved": ach,
+                "peak": mult * pk["bf16"], "unit": "TFLOP/s", "frac": ach / (mult * pk["bf16"]),
+                "peak_kind": pk["kind"] + (" bf16 burst" if mult == 1 else " bf16 burst x 2 (fp8 nominal ratio)"),
+                "peak_sustained": mult * pk["bf16_sustained"],
+                "frac_of_sustained": ach / (mult * pk["bf16_sustained"]),
                 "algorithmic_flops_per_launch": w13_flops}
-        if dt == 1:
-            roof["peak"] = 2 * peak_tf
-            roof["frac"] = roof["achieved"] / roof["peak"]
-            roof["peak_kind"] = peak_kind + " (bf16 sustained x 2, the nominal fp8/bf16 ratio)"
+        layer_frac = {"layer_tflops_frac_of_burst": flops / (ms_per_step * 1e-3) / 1e12 / (mult * pk["bf16"]),
+                      "layer_tflops_frac_of_sustained":
+                          flops / (ms_per_step * 1e-3) / 1e12 / (mult * pk["bf16_sustained"])}
     else:
         achieved = w13_bytes / w13_s / 1e9
         roof = {"kernel": "grouped_gemm_kernel<swap-AB, w13>", "bound": "hbm", "achieved": achieved,
-                "peak": peak, "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"], "peak_kind": pk["kind"],
                 "algorithmic_bytes_per_launch": w13_bytes}
-    roof.update({"traffic": kernel_traffic(args.workload), "kernel_us": 1e3 * w13_kernel_ms,
+        layer_frac = {}
+    roof.update({"traffic": kernel_traffic(name), "kernel_us": 1e3 * w13_kernel_ms,
                  "timed_by": "CUDA events recorded on the launch stream right before and after the "
                              "w13 GEMM, inside a graph of the layer, L2 flushed per step"})
-    line = {
-        "metric": "MoE layer tokens/s", "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8-e4m3" if dt == 1 else "bf16", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: {describe(wl)}", "global_batch": world * T,
-                   "active_experts": e_act, "l2": "flushed (256 MiB write) between timed steps",
-                   "parallelism": f"dp{world} (independent decode batches)",
-                   "mode": "batch_invariant" if args.batch_invariant else "default"},
+    res = {
+        "workload": f"{name}: {describe(wl)}",
+        "value": value, "unit": "tokens/s", "steps": steps, "ms_per_step": ms_per_step,
+        "dtype": "fp8-e4m3" if dt == 1 else "bf16", "active_experts": e_act,
         "us_per_layer": 1e3 * ms_per_step,
         "us_per_layer_p50": 1e3 * statistics.median(step_ms),
         "us_per_layer_direct_launch": 1e3 * direct_ms,
-        "timing": "per step: device time of one CUDA-graph replay of moe_forward (events on the "
-                  "stream around the replay); stages_us from a separate instrumented graph",
         "weight_bytes": weight_bytes,
         "weight_gbs": weight_bytes / (ms_per_step * 1e-3) / 1e9,
-        "weight_gbs_frac_of_measured_hbm": weight_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
+        "weight_gbs_frac_of_hbm_peak": weight_bytes / (ms_per_step * 1e-3) / 1e9 / pk["hbm"],
         "weight_gbs_frac_of_8tbs": weight_bytes / (ms_per_step * 1e-3) / 8e12,
-        "layer_tflops": 2.0 * T * k * 3 * I * H / (ms_per_step * 1e-3) / 1e12,
-        "all_bytes": all_bytes,
-        "all_gbs": all_bytes / (ms_per_step * 1e-3) / 1e9,
+        "layer_tflops": flops / (ms_per_step * 1e-3) / 1e12, **layer_frac,
+        "all_bytes": all_bytes, "all_gbs": all_bytes / (ms_per_step * 1e-3) / 1e9,
         "stages_us": {k_: 1e3 * v for k_, v in stage_ms.items()},
         "roofline": roof,
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                 "d2h_bytes_per_step": T * H * 2, "steps": e2e_steps},
-        "gpu_launches": launches_per_step(wl, T) * args.steps,
-        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step(wl, T) * steps,
+        "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and name == args.workload:
         host = host_copy(inp)
         toks = list(range(min(CPU_BASELINE_TOKENS, T)))
         secs = oracle_sample_seconds(host, wl, toks)
-        line["cpu_baseline"] = {"value": len(toks) / secs, "unit": "tokens/s", "cores": blas_threads(),
-                                "cpu": cpu_model(),
-                                "kind": "oracle",
-                                "sample": f"fp64 oracle on tokens 0..{len(toks) - 1} of the batch "
-                                          f"(routing of all {T} tokens), {secs:.1f} s"}
+        cpu = {"value": len(toks) / secs, "unit": "tokens/s", "cores": blas_threads(), "cpu": cpu_model(),
+               "kind": "oracle",
+               "sample": f"fp64 oracle on tokens 0..{len(toks) - 1} of the batch as a layer call of their own "
+                         f"(their routing, scales and expert products), {secs:.1f} s"}
+    del inp, ws, out, flush
+    torch.cuda.empty_cache()
+    return res, cpu
+
+
+def run_ours(args, wl, rank, world, local):
+    pk = peaks()
+    head, cpu = measure_workload(args.workload, wl, args, rank, world, local, steps_exact=args.steps)
+    nested = {}
+    if world == 1 and not args.only_headline:
+        for name in ORDER:
+            if name == args.workload:
+                nested[name] = head
+                continue
+            w = dict(WORKLOADS[name])
+            nested[name] = measure_workload(name, w, args, rank, world, local)[0]
+    line = {
+        "metric": "MoE layer tokens/s", "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": head["dtype"], "data": "synthetic",
+        "config": {"workload": head["workload"], "global_batch": world * wl["T"],
+                   "active_experts": head["active_experts"],
+                   "l2": "flushed (256 MiB write) between timed steps",
+                   "parallelism": f"dp{world} (independent batches)",
+                   "mode": "batch_invariant" if args.batch_invariant else "default"},
+        "timing": "per step: device time of one CUDA-graph replay of moe_forward (events on the "
+                  "stream around the replay); stages_us from a separate instrumented graph",
+        "peaks": pk,
+    }
+    for key in ("us_per_layer", "us_per_layer_p50", "us_per_layer_direct_launch", "weight_bytes", "weight_gbs",
+                "weight_gbs_frac_of_hbm_peak", "weight_gbs_frac_of_8tbs", "layer_tflops", "all_bytes",
+                "all_gbs", "stages_us", "roofline", "e2e", "gpu_launches", "clocks"):
+        line[key] = head[key]
+    if nested:
+        line["workloads"] = nested
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -497,10 +581,12 @@ def run_ours(args, wl, rank, world, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=None, help="timed steps (default 5000; reference: 5)")
-    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default 20; reference: 1)")
-    ap.add_argument("--workload", default="decode", choices=list(WORKLOADS))
+    ap.add_argument("--steps", type=int, default=None, help="timed steps of the headline (default 200; "
+                                                             "reference: 5)")
+    ap.add_argument("--warmup", type=int, default=None, help="warm-up steps (default 10; reference: 1)")
+    ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--only-headline", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch-invariant", action="store_true",
                     help="time moe_forward_batch_invariant (bf16 workloads)")
@@ -514,6 +600,8 @@ def main():
         wl["T"] = args.tokens
     if args.experts:
         wl["E"] = args.experts
+    if args.tokens or args.experts or args.batch_invariant:
+        args.only_headline = True
     if args.impl == "reference":
         # the fp64 oracle takes seconds per token: small defaults, one-token samples
         args.steps = 5 if args.steps is None else args.steps
@@ -522,8 +610,8 @@ def main():
         world = int(os.environ.get("WORLD_SIZE", "1"))
         run_reference(args, wl, rank, world)
         return
-    args.steps = 5000 if args.steps is None else args.steps
-    args.warmup = 20 if args.warmup is None else args.warmup
+    args.steps = 200 if args.steps is None else args.steps
+    args.warmup = 10 if args.warmup is None else args.warmup
     rank, world, local = dist_setup(args.gpus)
     try:
         run_ours(args, wl, rank, world, local)

@@ -37,11 +37,14 @@
  *    id out of range) are recorded in the workspace's status word and read
  *    with moe_get_status.
  *  - Repeated calls of moe_forward / moe_forward_batch_invariant (without
- *    debug outputs) or moe_forward_hostio with identical arguments are
- *    replayed from a CUDA graph the library records on the second such call
- *    (on an internal stream; nothing runs during the recording) and keeps
- *    for up to 32 argument sets.  Buffers are read at replay time.  Calls on
- *    a stream that is being captured always enqueue their kernels directly.
+ *    debug outputs) with identical arguments are replayed from a CUDA graph
+ *    the library records on the second such call (on an internal stream;
+ *    nothing runs during the recording) and keeps for up to 32 argument sets
+ *    per device.  Buffers are read at replay time.  Calls on a stream that is
+ *    being captured always enqueue their kernels directly.  A caller that
+ *    passes the same out and workspace buffers on every call benefits; a new
+ *    address is a new argument set.  moe_forward_hostio is never replayed
+ *    from a graph (its host buffers may not outlive the call).
  *  - Shapes are runtime values; nothing is specialised per T (the pages'
  *    lesson about per-token-count JIT recompiles, "AWS details MoE kernel
  *    fixes...", third fix).  Results are deterministic: identical inputs give
@@ -97,6 +100,8 @@ typedef struct {
   int inject_stall;    /* failure-path test: 1 makes the first gate/up GEMM CTA leave one
                           pipeline stage unfilled, so a bounded wait expires and the call
                           records MOE_ERR_DEVICE_TIMEOUT (the output is then undefined) */
+  uint8_t *hidden_q;   /* [T, H] FP8 path: the E4M3 codes of hidden / s1 that the gate/up
+                          GEMM consumed, in token order */
 } moe_debug_out_t;
 
 /* Bytes of workspace moe_forward needs for this shape (0 if the shape is
@@ -192,6 +197,13 @@ moe_status_t moe_align(const int32_t *topk_ids, int T, int E, int top_k, int32_t
 moe_status_t moe_route_static(const void *hidden, const void *router_w, const float *router_bias,
                               int T, int H, int E, int top_k, int32_t *topk_ids, float *topk_w,
                               void *stream);
+
+/* Counters of the launch cache since the library was loaded, for tests and
+ * diagnostics: out4[0] graph launches (replays), out4[1] graphs recorded,
+ * out4[2] recordings that failed (those calls ran directly), out4[3] calls
+ * that enqueued their kernels directly (first sightings, debug outputs,
+ * calls on a capturing stream).  out4 is host memory of 4 entries. */
+void moe_cache_stats(unsigned long long *out4);
 
 /* Synchronises `stream`, returns the first device-side error recorded in the
  * workspace since the last call (MOE_OK if none) and clears it.  *info_out

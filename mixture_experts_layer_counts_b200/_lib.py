@@ -24,7 +24,7 @@ STATUS = {
 # every symbol include/moe.h declares
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_forward", "moe_forward_hostio",
            "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static",
-           "moe_forward_batch_invariant")
+           "moe_forward_batch_invariant", "moe_cache_stats")
 
 
 class DebugOut(C.Structure):
@@ -33,6 +33,7 @@ class DebugOut(C.Structure):
         ("offsets", C.c_void_p), ("perm", C.c_void_p), ("inv_perm", C.c_void_p),
         ("inter", C.c_void_p), ("act_scales", C.c_void_p), ("stage_events", C.c_void_p),
         ("force_orient", C.c_int), ("wait_timeout_us", C.c_int), ("inject_stall", C.c_int),
+        ("hidden_q", C.c_void_p),
     ]
 
 
@@ -72,6 +73,8 @@ def lib() -> C.CDLL:
         L.moe_align.argtypes = [vp, i, i, i, vp, vp, vp, vp, vp, sz, vp]
         L.moe_get_status.restype = i
         L.moe_get_status.argtypes = [vp, vp, C.POINTER(C.c_uint32)]
+        L.moe_cache_stats.restype = None
+        L.moe_cache_stats.argtypes = [C.POINTER(C.c_ulonglong)]
         L.moe_status_string.restype = C.c_char_p
         L.moe_status_string.argtypes = [i]
         _lib = L

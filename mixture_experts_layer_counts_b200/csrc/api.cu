@@ -311,6 +311,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     MOE_TRY(cuda_status(cp(dbg->inter, L.inter, static_cast<size_t>(A) * I * (fp8 ? 1 : 2))));
     if (dbg->act_scales)
       MOE_TRY(cuda_status(cudaMemcpyAsync(dbg->act_scales, hdr + kHdrScaleS1, 8, cudaMemcpyDeviceToDevice, st)));
+    if (dbg->hidden_q && fp8)
+      MOE_TRY(cuda_status(launch_unpermute_rows(xperm, at<int32_t>(ws, L.inv_perm), T, k, H, dbg->hidden_q, st)));
   }
   return MOE_OK;
 }
@@ -326,13 +328,17 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
 // stream is being captured, and calls with debug outputs, run directly.  A
 // graph reads its buffers at replay time, so new contents at the same
 // addresses are seen; any change of pointer or size is a different key.
+// Only calls whose every pointer is device memory are cached (a graph would
+// keep host addresses in its copy nodes past the lifetime of the caller's
+// pinned buffers).  One cache per device; the capture and instantiation run
+// outside the cache's lock, so other threads are not held up by them (a call
+// that finds its key being captured by another thread runs directly).
 struct CallKey {
   int kind;
-  int dev;
   const void* p[9];
   long long n[7];
   bool operator==(const CallKey& o) const {
-    if (kind != o.kind || dev != o.dev) return false;
+    if (kind != o.kind) return false;
     for (int i = 0; i < 9; ++i)
       if (p[i] != o.p[i]) return false;
     for (int i = 0; i < 7; ++i)
@@ -341,72 +347,113 @@ struct CallKey {
   }
 };
 
+enum CacheState { kEmpty = 0, kSeenOnce = 1, kReady = 2, kFailed = 3, kCapturing = 4 };
+
 struct CacheEntry {
   CallKey key;
-  int state;               // 0 empty, 1 seen once, 2 graph ready, 3 capture failed
+  int state;
   cudaGraphExec_t exec;
   unsigned long long used;
 };
 
 constexpr int kCacheEntries = 32;
 
+struct DeviceCache {
+  std::mutex mu;
+  CacheEntry e[kCacheEntries];
+  cudaStream_t capture_stream = nullptr;
+  unsigned long long clock = 0;
+};
+
+struct CacheStats {
+  std::mutex mu;
+  unsigned long long replays = 0, captures = 0, failures = 0, direct = 0;
+};
+
+CacheStats& cache_stats() {
+  static CacheStats s;
+  return s;
+}
+
+void count(unsigned long long CacheStats::*field) {
+  CacheStats& s = cache_stats();
+  std::lock_guard<std::mutex> lock(s.mu);
+  ++(s.*field);
+}
+
 template <class Enqueue>
-moe_status_t run_cached(const CallKey& key, cudaStream_t st, Enqueue&& enqueue) {
-  static std::mutex mu;
-  static CacheEntry cache[kCacheEntries];
-  static cudaStream_t capture_stream[kMaxDevices] = {};
-  static unsigned long long clock = 0;
+moe_status_t run_direct(cudaStream_t st, Enqueue&& enqueue) {
+  count(&CacheStats::direct);
+  return enqueue(st);
+}
+
+template <class Enqueue>
+moe_status_t run_cached(int dev, const CallKey& key, cudaStream_t st, Enqueue&& enqueue) {
+  static DeviceCache caches[kMaxDevices];
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
-  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
-    return enqueue(st);
-  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= kMaxDevices || cudaStreamIsCapturing(st, &cs) != cudaSuccess ||
+      cs != cudaStreamCaptureStatusNone)
+    return run_direct(st, enqueue);
+  DeviceCache& c = caches[dev];
   CacheEntry* e = nullptr;
-  for (int i = 0; i < kCacheEntries; ++i)
-    if (cache[i].state != 0 && cache[i].key == key) e = &cache[i];
-  if (e == nullptr) {   // first sighting: remember the key, run directly
-    CacheEntry* v = &cache[0];
-    for (int i = 0; i < kCacheEntries; ++i) {
-      if (cache[i].state == 0) {
-        v = &cache[i];
-        break;
-      }
-      if (cache[i].used < v->used) v = &cache[i];
+  cudaStream_t cap = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < kCacheEntries; ++i)
+      if (c.e[i].state != kEmpty && c.e[i].key == key) e = &c.e[i];
+    if (e == nullptr) {   // first sighting: remember the key, run directly
+      CacheEntry* v = nullptr;
+      for (int i = 0; i < kCacheEntries && v == nullptr; ++i)
+        if (c.e[i].state == kEmpty) v = &c.e[i];
+      for (int i = 0; i < kCacheEntries && v == nullptr; ++i) v = &c.e[i];
+      for (int i = 0; i < kCacheEntries; ++i)   // least recently used, never one being captured
+        if (c.e[i].state != kCapturing && c.e[i].used < v->used) v = &c.e[i];
+      if (v->state == kCapturing) return run_direct(st, enqueue);
+      if (v->state == kReady) cudaGraphExecDestroy(v->exec);
+      *v = CacheEntry{key, kSeenOnce, nullptr, ++c.clock};
+      return run_direct(st, enqueue);
     }
-    if (v->state == 2) cudaGraphExecDestroy(v->exec);
-    *v = CacheEntry{key, 1, nullptr, ++clock};
-    return enqueue(st);
+    e->used = ++c.clock;
+    if (e->state == kReady) {
+      const cudaError_t err = cudaGraphLaunch(e->exec, st);
+      if (err == cudaSuccess) count(&CacheStats::replays);
+      return cuda_status(err);
+    }
+    if (e->state != kSeenOnce) return run_direct(st, enqueue);   // failed, or another thread captures
+    if (c.capture_stream == nullptr &&
+        cudaStreamCreateWithFlags(&c.capture_stream, cudaStreamNonBlocking) != cudaSuccess) {
+      c.capture_stream = nullptr;
+      e->state = kFailed;
+      count(&CacheStats::failures);
+      return run_direct(st, enqueue);
+    }
+    e->state = kCapturing;
+    cap = c.capture_stream;
   }
-  e->used = ++clock;
-  if (e->state == 3) return enqueue(st);
-  if (e->state == 1) {
-    if (key.dev < 0 || key.dev >= kMaxDevices) {
-      e->state = 3;
-      return enqueue(st);
-    }
-    if (capture_stream[key.dev] == nullptr &&
-        cudaStreamCreateWithFlags(&capture_stream[key.dev], cudaStreamNonBlocking) != cudaSuccess) {
-      capture_stream[key.dev] = nullptr;
-      e->state = 3;
-      return enqueue(st);
-    }
-    cudaStream_t cap = capture_stream[key.dev];
-    cudaGraph_t graph = nullptr;
-    bool ok = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
-    if (ok) {
-      const moe_status_t rc = enqueue(cap);
-      const cudaError_t end = cudaStreamEndCapture(cap, &graph);
-      ok = rc == MOE_OK && end == cudaSuccess && graph != nullptr;
-      if (ok) ok = cudaGraphInstantiate(&e->exec, graph, 0ULL) == cudaSuccess;
-      if (graph != nullptr) cudaGraphDestroy(graph);
-    }
-    cudaGetLastError();   // a failed capture leaves no sticky error
-    if (!ok) {
-      e->state = 3;
-      return enqueue(st);
-    }
-    e->state = 2;
+  // second sighting: record outside the lock (only this thread uses `cap`
+  // while the entry is marked as capturing, and an entry being captured is
+  // never evicted)
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  bool ok = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+  if (ok) {
+    const moe_status_t rc = enqueue(cap);
+    const cudaError_t end = cudaStreamEndCapture(cap, &graph);
+    ok = rc == MOE_OK && end == cudaSuccess && graph != nullptr;
+    if (ok) ok = cudaGraphInstantiate(&exec, graph, 0ULL) == cudaSuccess;
+    if (graph != nullptr) cudaGraphDestroy(graph);
   }
-  return cuda_status(cudaGraphLaunch(e->exec, st));
+  cudaGetLastError();   // a failed capture leaves no sticky error
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    e->state = ok ? kReady : kFailed;
+    e->exec = ok ? exec : nullptr;
+  }
+  count(ok ? &CacheStats::captures : &CacheStats::failures);
+  if (!ok) return run_direct(st, enqueue);
+  const cudaError_t err = cudaGraphLaunch(exec, st);
+  if (err == cudaSuccess) count(&CacheStats::replays);
+  return cuda_status(err);
 }
 
 int current_device() {
@@ -443,10 +490,9 @@ moe_status_t moe_forward(const void* hidden, const void* router_w, const float* 
                         top_k, dtype, out, workspace, workspace_bytes, dbg, s);
   };
   if (dbg != nullptr || check_shape(T, H, E, I, top_k, dtype) != MOE_OK) return enqueue(st);
-  const CallKey key{0, current_device(),
-                    {hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, out, workspace},
+  const CallKey key{0, {hidden, router_w, router_bias, w13, w2, w13_scale, w2_scale, out, workspace},
                     {T, H, E, I, top_k, dtype, static_cast<long long>(workspace_bytes)}};
-  return run_cached(key, st, enqueue);
+  return run_cached(current_device(), key, st, enqueue);
 }
 
 moe_status_t moe_forward_batch_invariant(const void* hidden, const void* router_w,
@@ -460,10 +506,9 @@ moe_status_t moe_forward_batch_invariant(const void* hidden, const void* router_
                         top_k, MOE_DTYPE_BF16, out, workspace, workspace_bytes, dbg, s, true);
   };
   if (dbg != nullptr || check_shape(T, H, E, I, top_k, MOE_DTYPE_BF16) != MOE_OK) return enqueue(st);
-  const CallKey key{1, current_device(),
-                    {hidden, router_w, router_bias, w13, w2, nullptr, nullptr, out, workspace},
+  const CallKey key{1, {hidden, router_w, router_bias, w13, w2, nullptr, nullptr, out, workspace},
                     {T, H, E, I, top_k, MOE_DTYPE_BF16, static_cast<long long>(workspace_bytes)}};
-  return run_cached(key, st, enqueue);
+  return run_cached(current_device(), key, st, enqueue);
 }
 
 moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
@@ -479,16 +524,13 @@ moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
   void* din = at<void>(workspace, L.staging_in);
   void* dout = at<void>(workspace, L.staging_out);
   const size_t bytes = static_cast<size_t>(T) * H * 2;
-  auto enqueue = [&](cudaStream_t s) {
-    MOE_TRY(cuda_status(cudaMemcpyAsync(din, hidden_host, bytes, cudaMemcpyHostToDevice, s)));
-    MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
-                         dtype, dout, workspace, workspace_bytes, nullptr, s));
-    return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, s));
-  };
-  const CallKey key{2, current_device(),
-                    {hidden_host, router_w, router_bias, w13, w2, w13_scale, w2_scale, out_host, workspace},
-                    {T, H, E, I, top_k, dtype, static_cast<long long>(workspace_bytes)}};
-  return run_cached(key, st, enqueue);
+  // Enqueued directly, never replayed from a cached graph: a graph would hold
+  // the host addresses in its copy nodes, and a later buffer at the same
+  // address need not be pinned.
+  MOE_TRY(cuda_status(cudaMemcpyAsync(din, hidden_host, bytes, cudaMemcpyHostToDevice, st)));
+  MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
+                       dtype, dout, workspace, workspace_bytes, nullptr, st));
+  return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
 }
 
 moe_status_t moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,
@@ -525,6 +567,16 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t
                at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots,
                at<int>(workspace, L.slice_hist)};
   return cuda_status(launch_align(aa, static_cast<cudaStream_t>(stream)));
+}
+
+void moe_cache_stats(unsigned long long* out4) {
+  if (!out4) return;
+  CacheStats& s = cache_stats();
+  std::lock_guard<std::mutex> lock(s.mu);
+  out4[0] = s.replays;
+  out4[1] = s.captures;
+  out4[2] = s.failures;
+  out4[3] = s.direct;
 }
 
 moe_status_t moe_get_status(void* workspace, void* stream, uint32_t* info_out) {

@@ -157,6 +157,30 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
   }
 }
 
+// Debug output: dst[t] = src[inv_perm[t * k]] (the first slot's copy of a
+// token row in perm order back in token order), 16-byte vectors.
+__global__ void unpermute_rows_kernel(const uint4* __restrict__ src, const int32_t* __restrict__ inv_perm,
+                                      int T, int k, int vpr, uint4* __restrict__ dst) {
+  const size_t n = static_cast<size_t>(T) * vpr;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / vpr);
+    const int c = static_cast<int>(i - static_cast<size_t>(t) * vpr);
+    const int p = inv_perm[static_cast<size_t>(t) * k];
+    if (p >= 0 && p < T * k) dst[i] = src[static_cast<size_t>(p) * vpr + c];
+  }
+}
+
+cudaError_t launch_unpermute_rows(const void* src, const int32_t* inv_perm, int T, int k, int row_bytes,
+                                  void* dst, cudaStream_t st) {
+  const int vpr = row_bytes / 16;
+  const size_t n = static_cast<size_t>(T) * vpr;
+  const int grid = static_cast<int>(std::min<size_t>((n + 255) / 256, static_cast<size_t>(sm_count()) * 4));
+  unpermute_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(src), inv_perm, T, k, vpr,
+                                              static_cast<uint4*>(dst));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int A, int k, int H,
                           bool fp8, const uint32_t* hdr, void* xperm, cudaStream_t st) {
   const int vpr = H / 8;

@@ -86,6 +86,10 @@ cudaError_t launch_align(const AlignArgs& a, cudaStream_t st);
 cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int A, int k, int H,
                           bool fp8, const uint32_t* hdr, void* xperm, cudaStream_t st);
 
+// Debug output: dst[t, :] = src[inv_perm[t * k], :] for rows of row_bytes (a multiple of 16)
+cudaError_t launch_unpermute_rows(const void* src, const int32_t* inv_perm, int T, int k, int row_bytes,
+                                  void* dst, cudaStream_t st);
+
 // FP8: s2 = max(amax_cta[0..n)) / 448, inter = E4M3(h32 / s2)
 cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
                            uint32_t* hdr, uint8_t* inter, cudaStream_t st);

@@ -83,7 +83,8 @@ extern "C" moe_status_t moe_route_static(const void* hidden, const void* router_
     return MOE_ERR_INVALID_ARG;
   if (T < 1 || H < 128 || H > 8192 || H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!hidden || !router_w || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  if ((reinterpret_cast<uintptr_t>(hidden) & 15u) || (reinterpret_cast<uintptr_t>(router_w) & 15u))
+  if ((reinterpret_cast<uintptr_t>(hidden) & 15u) || (reinterpret_cast<uintptr_t>(router_w) & 15u) ||
+      (reinterpret_cast<uintptr_t>(router_bias) & 3u))   // the bias is read as fp32
     return MOE_ERR_MISALIGNED;
   if (static_cast<long long>(T) * E > (1LL << 24)) return MOE_ERR_EXCEEDS_STATIC_SCRATCH;
   const StaticRouteLayout L = static_route_layout(T, E);

@@ -65,7 +65,8 @@ def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w
     """out[T, H] bf16 of the fused MoE layer (see include/moe.h).
 
     ``debug``: optional dict; keys filled on return (device tensors):
-    topk_ids, topk_w, counts, offsets, perm, inv_perm, inter, act_scales.
+    topk_ids, topk_w, counts, offsets, perm, inv_perm, inter, act_scales and,
+    on the FP8 path, hidden_q (the E4M3 codes of hidden / s1).
     ``stage_events``: optional list of 8 torch.cuda.Event recorded at the
     stage boundaries on the launch stream.
     ``batch_invariant``: call moe_forward_batch_invariant (bf16 only): each
@@ -104,7 +105,11 @@ def moe_forward(hidden, router_w, router_bias, w13, w2, top_k, w13_scale=None, w
             debug["inter"] = torch.empty((A, I), dtype=torch.bfloat16 if dt == MOE_DTYPE_BF16 else torch.uint8,
                                          device=dev)
             debug["act_scales"] = torch.zeros(2, dtype=torch.float32, device=dev)
-            for k in ("topk_ids", "topk_w", "counts", "offsets", "perm", "inv_perm", "inter", "act_scales"):
+            names = ["topk_ids", "topk_w", "counts", "offsets", "perm", "inv_perm", "inter", "act_scales"]
+            if dt == MOE_DTYPE_FP8_E4M3:
+                debug["hidden_q"] = torch.empty((T, H), dtype=torch.uint8, device=dev)
+                names.append("hidden_q")
+            for k in names:
                 setattr(dbg, k, debug[k].data_ptr())
         if stage_events is not None:
             arr = (C.c_void_p * N_STAGE_EVENTS)(

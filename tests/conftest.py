@@ -19,3 +19,18 @@ def cuda_ok():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return True
+
+
+def pytest_sessionfinish(session, exitstatus):
+    # parity records (strict-bound ratios, envelope use, FP8 code agreement)
+    path = os.environ.get("MOE_PARITY_LOG")
+    if not path:
+        return
+    try:
+        import json
+
+        from helpers import PARITY_LOG
+    except Exception:
+        return
+    with open(path, "w") as f:
+        json.dump(PARITY_LOG, f, indent=1)

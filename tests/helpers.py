@@ -130,7 +130,25 @@ def assert_inter_equal(dbg, ref, amb):
     return n_diff, n_amb
 
 
+# Parity records of the tests that run (written to $MOE_PARITY_LOG at the end
+# of the session when that variable is set; see conftest.py).
+PARITY_LOG = []
+
+
+def _current_test():
+    import os
+    return os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+
+
 def assert_output_close(out, ref, fp8, tokens=None, env=None):
+    """Output acceptance against the oracle.
+
+    bf16: |gpu - ref| <= 2e-2 |ref| + 2e-3 rms(ref) per element, rms over the
+    compared elements.  Only a test that passes ``env`` (the output change the
+    alternative correct roundings of the intermediate can cause, from
+    bf16_rounding_ambiguity) may widen that bound by env, and every element
+    that needed it is counted in the parity log.  FP8: relative L2 <= 3e-2.
+    """
     o = out.float().cpu().numpy().astype(np.float64)
     r = ref["out"]
     if tokens is not None:
@@ -138,8 +156,85 @@ def assert_output_close(out, ref, fp8, tokens=None, env=None):
         env = None if env is None else env[tokens]
     if fp8:
         err = rel_l2(o, r)
+        PARITY_LOG.append(dict(test=_current_test(), kind="fp8", rel_l2=err))
         assert err <= 3e-2, f"FP8 relative L2 {err:.4g} > 3e-2"
         return err
-    v = bf16_tolerance_violation(o, r, extra=env)
+    v = bf16_tolerance_violation(o, r)
+    rec = dict(test=_current_test(), kind="bf16", strict_ratio=v, n_over_strict=0, env_used=False)
+    if v > 1.0 and env is not None:
+        rms = float(np.sqrt(np.mean(r * r)))
+        bound = 2e-2 * np.abs(r) + 2e-3 * rms
+        over = np.abs(o - r) > bound
+        rec.update(n_over_strict=int(over.sum()), n_elements=int(o.size), env_used=True,
+                   max_env_over_bound=float((env / bound).max()),
+                   ratio_with_env=bf16_tolerance_violation(o, r, extra=env))
+        PARITY_LOG.append(rec)
+        assert rec["ratio_with_env"] <= 1.0, f"bf16 tolerance exceeded even with the rounding envelope: {rec}"
+        return v
+    PARITY_LOG.append(rec)
     assert v <= 1.0, f"bf16 tolerance exceeded: worst ratio {v:.3g}"
     return v
+
+
+def fp8_intermediate_check(dbg, inp, ref, s2_gpu):
+    """The GPU's E4M3 intermediate codes against the oracle's h.
+
+    The GPU forms h in fp32 from fp32 accumulations of exact E4M3 products and
+    quantises fl32(h / s2) with round-to-nearest-even; where the exact h / s2
+    is farther from an E4M3 rounding boundary than that arithmetic can move
+    it, the code is unique and must equal E4M3(h / s2).  Band of the kernel's
+    h (as in bf16_rounding_ambiguity, with a wider accumulation term for the
+    long E4M3 reductions): 2^-19 |h| + 2^-17 (|SiLU'(g) u| S_g + |SiLU(g)| S_u).
+    Returns (codes compared, codes that differ from E4M3(h_ref / s2_gpu),
+    codes inside the ambiguous band).
+    """
+    from scipy.special import expit
+
+    from mixture_experts_layer_counts_b200.inputs import host_bits as hb
+    from oracle import decode_weight, e4m3_code_to_f64, round_to_e4m3_satfinite
+
+    k = inp["top_k"]
+    xq = e4m3_code_to_f64(ref["xq"]) * np.float64(ref["s1"])
+    perm, off = ref["perm"], ref["offsets"]
+    gi = e4m3_code_to_f64(hb(dbg["inter"]))
+    s13 = inp["w13_scale"].cpu().numpy()
+    n = n_diff = n_amb = 0
+    for e in range(len(off) - 1):
+        rows = list(range(off[e], off[e + 1]))
+        if not rows:
+            continue
+        W = decode_weight(hb(inp["w13"][e]), s13[e])
+        I = W.shape[0] // 2
+        Xe = xq[perm[rows] // k]
+        g, u = Xe @ W[:I].T, Xe @ W[I:].T
+        Sg, Su = np.abs(Xe) @ np.abs(W[:I]).T, np.abs(Xe) @ np.abs(W[I:]).T
+        sig = expit(g)
+        sl = g * sig
+        ds = sig * (1.0 + g * (1.0 - sig))
+        h = sl * u
+        band = 2.0 ** -19 * np.abs(h) + 2.0 ** -17 * (np.abs(ds * u) * Sg + np.abs(sl) * Su)
+        s2 = np.float64(s2_gpu)
+        c = round_to_e4m3_satfinite(h / s2)
+        lo = round_to_e4m3_satfinite((h - band) / s2)
+        hi = round_to_e4m3_satfinite((h + band) / s2)
+        got = gi[rows]
+        ok = (got >= lo) & (got <= hi)
+        assert ok.all(), f"expert {e}: E4M3 intermediate codes outside their valid range"
+        n += got.size
+        n_diff += int((got != c).sum())
+        n_amb += int((lo != hi).sum())
+    PARITY_LOG.append(dict(test=_current_test(), kind="fp8_inter", codes=n, differ=n_diff, ambiguous=n_amb))
+    return n, n_diff, n_amb
+
+
+def assert_fp8_scales_and_codes(dbg, inp, ref):
+    """s1 bit-exact, hidden_q bit-exact, s2 within the fp32 arithmetic of its
+    amax, intermediate codes per fp8_intermediate_check."""
+    from mixture_experts_layer_counts_b200.inputs import host_bits as hb
+
+    sc = dbg["act_scales"].cpu().numpy()
+    assert sc[0] == np.float32(ref["s1"]), "activation scale s1 differs"
+    assert np.array_equal(hb(dbg["hidden_q"]), ref["xq"]), "E4M3 activation codes differ"
+    rel = abs(float(sc[1]) - float(ref["s2"])) / float(ref["s2"])
+    assert rel <= 2.0 ** -16, f"intermediate scale s2 {sc[1]} vs {ref['s2']}"
+    return fp8_intermediate_check(dbg, inp, ref, sc[1])

@@ -7,7 +7,6 @@ MOE_ERR_DEVICE_TIMEOUT in the workspace status word, drains what it issued,
 frees its tensor memory and returns.  The host reads the status; the context
 stays usable and the next call on the same workspace is correct.
 """
-import numpy as np
 import pytest
 import torch
 
@@ -35,5 +34,7 @@ def test_bounded_wait_reports_timeout_and_recovers(cuda_ok):
     assert layer.get_status(ws)[0] == 0            # cleared once read
     out = _call(inp, ws)                            # same workspace, no injection
     assert layer.get_status(ws)[0] == 0
+    fresh = _call(inp, layer.make_workspace(T, H, E, I, k, 0))
+    assert torch.equal(out.view(torch.int16), fresh.view(torch.int16))   # as if nothing had failed
     ref = oracle_of(inp)
-    assert_output_close(out, ref, fp8=False, env=np.full_like(ref["out"], 1e-3))
+    assert_output_close(out, ref, fp8=False)        # the stated bf16 bound
