@@ -161,6 +161,43 @@ moe_status_t moe_forward_hostio(const void *hidden_host, const void *router_w,
                                 int E, int I, int top_k, int dtype, void *out_host,
                                 void *workspace, size_t workspace_bytes, void *stream);
 
+/* Tensor parallelism over the intermediate dimension I.  The pages' serving
+ * figures come from 8-way tensor-parallel deployments ("AWS details MoE kernel
+ * fixes for SageMaker, upstreams them to vLLM", The facts); for this layer the
+ * split that stays balanced under skewed routing is over I: rank g of G holds
+ * rows [g I/G, (g+1) I/G) of every expert's gate and up projections and the
+ * matching columns of its down projection, so every rank streams 1/G of
+ * every active expert.  h = SiLU(g) * u of an intermediate column depends
+ * only on that column's gate and up rows, so the bf16 intermediate is the
+ * same as without the split; the output is the sum over ranks of
+ *   partial_g[t] = sum_j w[t, j] * W2[e][:, slice g] h[slice g].
+ *
+ * moe_forward_partial: the layer on one rank's slice.  Same arguments and
+ * errors as moe_forward, with
+ *   w13_shard [E, 2 * I_shard, H]: rows [0, I_shard) this rank's gate rows,
+ *             rows [I_shard, 2 * I_shard) its up rows (bf16 or E4M3)
+ *   w2_shard  [E, H, I_shard]: the matching columns of w2
+ *   out_partial [T, H] fp32 (device): the unrounded slot-ordered sum above
+ *   workspace >= moe_workspace_size(T, H, E, I_shard, top_k, dtype)
+ * Routing is computed on every rank from the replicated hidden and router
+ * weights; it is deterministic, so every rank routes identically.  FP8: the
+ * activation scale s1 is the same on every rank; the intermediate scale s2
+ * is taken over this rank's slice of h (a scale per shard, not per tensor).
+ *
+ * moe_sum_partials: out[t, :] = bf16( sum_{g=0..G-1} partials[g, t, :] ),
+ * the fp32 partials added in rank order from g = 0 and rounded once, so
+ * every rank that holds the gathered partials [G, T, H] (fp32, device)
+ * computes the same bits.  out [T, H] bf16 (device).  The exchange of the
+ * partials between ranks (an all-gather into local memory) is the caller's
+ * collective. */
+moe_status_t moe_forward_partial(const void *hidden, const void *router_w, const float *router_bias,
+                                 const void *w13_shard, const void *w2_shard, const float *w13_scale,
+                                 const float *w2_scale, int T, int H, int E, int I_shard, int top_k,
+                                 int dtype, float *out_partial, void *workspace, size_t workspace_bytes,
+                                 void *stream);
+
+moe_status_t moe_sum_partials(const float *partials, int G, int T, int H, void *out, void *stream);
+
 /* Router only: topk_ids [T, top_k] int32 and topk_w [T, top_k] fp32 (device),
  * same definition as in moe_forward.  Uses the workspace of moe_forward's
  * shape (moe_workspace_size with the same T, H, E, top_k; any I >= 128). */

@@ -24,7 +24,7 @@ STATUS = {
 # every symbol include/moe.h declares
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_forward", "moe_forward_hostio",
            "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static",
-           "moe_forward_batch_invariant", "moe_cache_stats")
+           "moe_forward_batch_invariant", "moe_cache_stats", "moe_forward_partial", "moe_sum_partials")
 
 
 class DebugOut(C.Structure):
@@ -65,6 +65,10 @@ def lib() -> C.CDLL:
         L.moe_forward_batch_invariant.argtypes = [vp] * 5 + [i] * 5 + [vp, vp, sz, vp, vp]
         L.moe_forward_hostio.restype = i
         L.moe_forward_hostio.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, vp]
+        L.moe_forward_partial.restype = i
+        L.moe_forward_partial.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, vp]
+        L.moe_sum_partials.restype = i
+        L.moe_sum_partials.argtypes = [vp, i, i, i, vp, vp]
         L.moe_route.restype = i
         L.moe_route.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, sz, vp]
         L.moe_route_static.restype = i

@@ -214,6 +214,7 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
     a.hdr[kHdrChunksSwap] = static_cast<uint32_t>(tsw);
     a.hdr[kHdrChunksNormal] = static_cast<uint32_t>(tno);
     a.hdr[kHdrChunksPair] = static_cast<uint32_t>(tpr);
+    a.hdr[kHdrBarrier] = 0u;   // arrival counter of the gate/up GEMM's closing grid barrier
   }
 
   // FP8 activation scale: s1 = amax / 448 (one IEEE fp32 division); amax == 0 -> 1

@@ -157,7 +157,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                           const void* w13, const void* w2, const float* w13_scale,
                           const float* w2_scale, int T, int H, int E, int I, int k, int dtype,
                           void* out, void* ws, size_t ws_bytes, moe_debug_out_t* dbg,
-                          cudaStream_t st, bool invariant = false) {
+                          cudaStream_t st, bool invariant = false, bool out_fp32 = false) {
   MOE_TRY(check_shape(T, H, E, I, k, dtype));
   const bool fp8 = dtype == MOE_DTYPE_FP8_E4M3;
   if (invariant && fp8) return MOE_ERR_INVALID_ARG;   // per-tensor FP8 scales span the batch
@@ -203,7 +203,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 router_bias, T, H, E, k,
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
-                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0};
+                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0,
+                at<int>(ws, L.tickets)};
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
@@ -241,6 +242,15 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g13.inject_stall = dbg ? dbg->inject_stall : 0;
   g13.whole_units = invariant ? 1 : 0;
   float* amax_cta = at<float>(ws, L.amax_cta);
+  // FP8: the last gate/up launch of the call requantises the whole
+  // intermediate after a grid barrier (per-tensor s2 over every launch's amax)
+  const int n_amax = (any_swap ? grid : 0) + (any_normal ? grid : 0);
+  auto requant_args = [&](GemmArgs& g, bool last) {
+    g.amax_all = amax_cta;
+    g.amax_n = (fp8 && last) ? n_amax : 0;
+    g.inter_q = inter;
+    g.requant_n4 = static_cast<long long>(A) * I / 4;
+  };
   if (any_swap) {
     GemmArgs g = g13;
     g.chunks = at<int4>(ws, L.chunks_swap);
@@ -248,6 +258,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.mtiles = I / kTileM;
     g.amax_cta = amax_cta;
     g.flags = flags + 0 * kMaxSlots;
+    requant_args(g, !any_normal);
     MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW13, fp8, tw13s, txs, g, grid, st)));
   }
   if (any_normal) {
@@ -257,14 +268,10 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
     g.amax_cta = amax_cta + (any_swap ? grid : 0);
     g.flags = flags + 1 * kMaxSlots;
+    requant_args(g, true);
     MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
   }
-  record(dbg, 4, st);
-  if (fp8) {
-    const int n_cta = (any_swap ? grid : 0) + (any_normal ? grid : 0);
-    MOE_TRY(cuda_status(launch_requant(at<float>(ws, L.h32), amax_cta, n_cta,
-                                       static_cast<size_t>(A) * I, hdr, static_cast<uint8_t*>(inter), st)));
-  }
+  record(dbg, 4, st);   // (the FP8 requantisation ran at the end of the gate/up GEMM)
   record(dbg, 5, st);
 
   GemmArgs g2 = g13;
@@ -276,7 +283,12 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g2.wscale = w2_scale;
   g2.act_scale = hdr + kHdrScaleS2;
   g2.amax_cta = nullptr;
+  g2.amax_n = 0;
   g2.inject_stall = 0;
+  g2.tickets = at<int>(ws, L.tickets);   // zeroed by the router's top-k kernel
+  g2.y_out = out;
+  g2.y_fp32 = out_fp32 ? 1 : 0;
+  g2.top_k = k;
   if (any_swap) {
     GemmArgs g = g2;
     g.chunks = at<int4>(ws, L.chunks_swap);
@@ -293,8 +305,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.flags = flags + 3 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
   }
-  record(dbg, 6, st);
-  MOE_TRY(cuda_status(launch_combine(at<float>(ws, L.ysc), T, k, H, static_cast<__nv_bfloat16*>(out), st)));
+  record(dbg, 6, st);   // the combine runs inside the down-projection GEMM's epilogue
   record(dbg, 7, st);
 
   if (dbg) {
@@ -531,6 +542,24 @@ moe_status_t moe_forward_hostio(const void* hidden_host, const void* router_w,
   MOE_TRY(forward_impl(din, router_w, router_bias, w13, w2, w13_scale, w2_scale, T, H, E, I, top_k,
                        dtype, dout, workspace, workspace_bytes, nullptr, st));
   return cuda_status(cudaMemcpyAsync(out_host, dout, bytes, cudaMemcpyDeviceToHost, st));
+}
+
+moe_status_t moe_forward_partial(const void* hidden, const void* router_w, const float* router_bias,
+                                 const void* w13_shard, const void* w2_shard, const float* w13_scale,
+                                 const float* w2_scale, int T, int H, int E, int I_shard, int top_k,
+                                 int dtype, float* out_partial, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  return forward_impl(hidden, router_w, router_bias, w13_shard, w2_shard, w13_scale, w2_scale, T, H, E,
+                      I_shard, top_k, dtype, out_partial, workspace, workspace_bytes, nullptr,
+                      static_cast<cudaStream_t>(stream), false, true);
+}
+
+moe_status_t moe_sum_partials(const float* partials, int G, int T, int H, void* out, void* stream) {
+  if (!partials || !out) return MOE_ERR_INVALID_ARG;
+  if (G < 1 || T < 1 || H < 128 || H > 8192 || H % 128 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(partials) || !aligned16(out)) return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_sum_partials(partials, G, static_cast<long long>(T) * H,
+                                         static_cast<__nv_bfloat16*>(out), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,

@@ -2,8 +2,6 @@
 //   gather   x_perm[p] = hidden[perm[p] / k]  (bf16), or its per-tensor E4M3
 //            quantisation x / s1 (FP8 path; one IEEE fp32 division, RNE,
 //            saturating to +-448)
-//   requant  FP8 intermediate: s2 = max(per-CTA amax|h|) / 448, h_q = E4M3(h / s2)
-//   combine  out[t] = bf16(sum_{j<k} ysc[t*k + j]) in slot order, fp32 sum
 // All grids are sized from the SM count; 16-byte vector accesses.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -90,71 +88,32 @@ __global__ void gather_quant_kernel(const uint4* __restrict__ hidden, const int3
   }
 }
 
-__global__ void requant_kernel(const float4* __restrict__ h32, const float* __restrict__ amax_cta,
-                               int n_cta, size_t n4, uint32_t* __restrict__ hdr,
-                               uint32_t* __restrict__ out) {
-  pdl_wait();
-  pdl_launch_next();
-  __shared__ float s_scale;
-  if (threadIdx.x < 32) {
-    float m = 0.f;
-    for (int i = threadIdx.x; i < n_cta; i += 32) m = fmaxf(m, amax_cta[i]);
-#pragma unroll
-    for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
-    if (threadIdx.x == 0) {
-      const float s2 = m == 0.f ? 1.0f : __fdiv_rn(m, 448.0f);
-      s_scale = s2;
-      if (blockIdx.x == 0) hdr[kHdrScaleS2] = __float_as_uint(s2);
+// Tensor-parallel sum: out[i] = bf16(parts[0][i] + parts[1][i] + ... ), the
+// partials added in rank order from the first, one rounding at the end.
+__global__ void __launch_bounds__(256) sum_partials_kernel(const float4* __restrict__ parts, int G,
+                                                           long long n4, uint2* __restrict__ out) {
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float4 acc = parts[i];
+    for (int g = 1; g < G; ++g) {
+      const float4 v = parts[static_cast<long long>(g) * n4 + i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
-  }
-  __syncthreads();
-  const float s2 = s_scale;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const float4 v = h32[i];
-    out[i] = pack_e4m3x4(__fdiv_rn(v.x, s2), __fdiv_rn(v.y, s2), __fdiv_rn(v.z, s2),
-                         __fdiv_rn(v.w, s2));
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    out[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
   }
 }
 
-// Work unit = (token t, block of 256 float4 columns); per thread the k slot
-// loads are issued together and summed in slot order.
-__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ ysc, int T, int k,
-                                                      int h4, uint2* __restrict__ out) {
-  pdl_wait();
-  pdl_launch_next();
-  const int nb = (h4 + 255) / 256;
-  const int units = T * nb;
-  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
-    const int t = unit / nb;
-    const int c = (unit - t * nb) * 256 + threadIdx.x;
-    if (c >= h4) continue;
-    const float4* src = ysc + static_cast<size_t>(t) * k * h4 + c;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      float4 y[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (j0 + u < k) y[u] = __ldcg(src + static_cast<size_t>(j0 + u) * h4);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (j0 + u < k) {
-          if (j0 + u == 0) {
-            acc = y[u];
-          } else {
-            acc.x += y[u].x;
-            acc.y += y[u].y;
-            acc.z += y[u].z;
-            acc.w += y[u].w;
-          }
-        }
-      }
-    }
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    out[static_cast<size_t>(t) * h4 + c] =
-        make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-  }
+cudaError_t launch_sum_partials(const float* parts, int G, long long n, __nv_bfloat16* out, cudaStream_t st) {
+  const long long n4 = n / 4;
+  const int grid = static_cast<int>(std::min<long long>((n4 + 255) / 256, static_cast<long long>(sm_count()) * 8));
+  sum_partials_kernel<<<grid > 0 ? grid : 1, 256, 0, st>>>(reinterpret_cast<const float4*>(parts), G, n4,
+                                                          reinterpret_cast<uint2*>(out));
+  return cudaGetLastError();
 }
 
 // Debug output: dst[t] = src[inv_perm[t * k]] (the first slot's copy of a
@@ -194,23 +153,6 @@ cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int 
                       reinterpret_cast<uint2*>(xperm));
   return launch_pdl(gather_kernel, dim3(ggrid), dim3(256), 0, st, reinterpret_cast<const uint4*>(hidden),
                     perm, A, k, vpr, reinterpret_cast<uint4*>(xperm));
-}
-
-cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
-                           uint32_t* hdr, uint8_t* inter, cudaStream_t st) {
-  const size_t n4 = count / 4;
-  const int grid = static_cast<int>(std::min<size_t>((n4 + 255) / 256, static_cast<size_t>(sm_count()) * 8));
-  return launch_pdl(requant_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(h32),
-                    amax_cta, n_cta, n4, hdr, reinterpret_cast<uint32_t*>(inter));
-}
-
-cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
-                           cudaStream_t st) {
-  const int h4 = H / 4;
-  const int units = T * ((h4 + 255) / 256);
-  const int grid = std::min(units, sm_count() * 8);
-  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(ysc), T,
-                    k, h4, reinterpret_cast<uint2*>(out));
 }
 
 }  // namespace moe

@@ -21,10 +21,15 @@
 //          adjacent gate and up tiles), so one thread holds g and u of the
 //          same (token, i) and the epilogue forms h = SiLU(g) * u directly:
 //          bf16 path -> inter (bf16, RNE); FP8 path -> h (fp32) + per-CTA
-//          amax|h| for the per-tensor requantisation that follows.
+//          amax|h|, and the last gate/up launch of the call closes with a
+//          grid barrier and the per-tensor E4M3 requantisation of h
+//          (requant_tail), so no separate pass is launched.
 //   kW2  : one accumulator; the epilogue multiplies by the router weight
-//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), which
-//          the combine pass sums in slot order: deterministic, no atomics.
+//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), then
+//          takes an integer ticket per (token, 128-column tile); the CTA that
+//          writes a token's last slot of a tile sums the k slot rows in slot
+//          order and writes the bf16 output (combine_tile): the combine runs
+//          inside this kernel, deterministic, no floating-point atomics.
 //
 // Work split.  A "unit" is one output tile (token chunk x weight-row tile)
 // and needs `katoms` K atoms.
@@ -59,6 +64,7 @@
 // tiles fill all 512 columns.  Every wait is bounded (see mbar_wait).
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include <cstdlib>
 
@@ -96,14 +102,18 @@ struct Cfg {
   static constexpr int kEpiCols = 16;
   static constexpr int kEpiLd = 20;
   static constexpr int kEpiBytes = kSwap ? 0 : kEpiWarps * 32 * kEpiLd * 4;
-  static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes) / kStageBytes;
+  // w2: two lists (units alternate) of the (token, tile) pairs whose combine
+  // this CTA completes, at most 2 * kTileM per unit, plus their lengths
+  static constexpr int kCombList = 2 * kTileM;
+  static constexpr int kCombBytes = kDual ? 0 : 2 * (kCombList + 4) * 4;
+  static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes - kCombBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kNumAcc = kDual ? 2 : 1;
   static constexpr int kAccCols = kNumAcc * kBN * (kPair ? 2 : 1);   // per TMEM buffer
   static constexpr int kAccBufs = kPair ? 1 : 2;               // pair: 512 columns, one buffer
   static constexpr int kTmemCols = kAccBufs * kAccCols;        // 128, 256 or 512
   static constexpr int kSmemBytes =
-      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes;
+      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes + kCombBytes;
   static constexpr int kAtomElems = FP8 ? 128 : 64;
   static constexpr int kSlotFloats = kNumAcc * kTileM * kBN;   // one CTA's partial tile
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
@@ -210,6 +220,103 @@ __device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, 
   }
 }
 
+__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// Combine of one (token t, ticket tile) pair by one warp: out[t, tile cols] =
+// bf16( sum_{j < k} ysc[t*k + j, tile cols] ), the fp32 sum in slot order
+// j = 0, 1, ... (the definition's order), 4 columns per lane.  The slot rows
+// were written by other CTAs: read through L2.
+__device__ __forceinline__ void combine_tile(const GemmArgs& a, int t, int tile, int lane) {
+  const int H = a.ld_out;
+  const int col = tile * kTicketCols + lane * 4;
+  const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.out) +
+                                                      static_cast<size_t>(t) * a.top_k * H + col);
+  const size_t stride = static_cast<size_t>(H) / 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j0 = 0; j0 < a.top_k; j0 += 8) {
+    float4 y[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (j0 + u < a.top_k) y[u] = __ldcg(src + static_cast<size_t>(j0 + u) * stride);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (j0 + u < a.top_k) {
+        if (j0 + u == 0) {
+          acc = y[u];
+        } else {
+          acc.x += y[u].x;
+          acc.y += y[u].y;
+          acc.z += y[u].z;
+          acc.w += y[u].w;
+        }
+      }
+    }
+  }
+  if (a.y_fp32) {   // tensor-parallel partial: the unrounded sum
+    *reinterpret_cast<float4*>(static_cast<float*>(a.y_out) + static_cast<size_t>(t) * H + col) = acc;
+    return;
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.y_out) + static_cast<size_t>(t) * H + col) =
+      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+}
+
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// Closing step of the last FP8 gate/up launch of a call: the per-tensor
+// requantisation of the intermediate.  Every CTA of the grid arrives at a
+// grid barrier once its epilogue stores and its amax|h| slot are written
+// (fence, then an integer arrival count); then each CTA forms
+// s2 = max(amax slots) / 448 (one IEEE fp32 division; amax 0 gives 1) and
+// writes E4M3(h / s2), round-to-nearest-even and saturating to +-448, for a
+// grid-strided part of the intermediate.  The wait is bounded: on expiry the
+// status word records it and the CTA returns without requantising.
+__device__ __forceinline__ void requant_tail(const GemmArgs& a, float* s_s2, volatile int* s_ok) {
+  __threadfence();   // this thread's stores of h (and amax) are visible device-wide
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    atomicAdd(a.hdr + kHdrBarrier, 1u);
+    const unsigned int need = gridDim.x;
+    bool ok = true;
+    if (ld_acquire(reinterpret_cast<const int*>(a.hdr + kHdrBarrier)) < static_cast<int>(need)) {
+      const uint64_t t0 = globaltimer_ns();
+      for (uint32_t it = 1;; ++it) {
+        if (ld_acquire(reinterpret_cast<const int*>(a.hdr + kHdrBarrier)) >= static_cast<int>(need)) break;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > a.timeout_ns) {
+          report_status(a.hdr, MOE_DEVICE_TIMEOUT, kSiteGridBarrier);
+          ok = false;
+          break;
+        }
+      }
+    }
+    float m = 0.f;
+    for (int i = 0; ok && i < a.amax_n; ++i) m = fmaxf(m, __ldcg(a.amax_all + i));
+    const float s2 = m == 0.f ? 1.0f : __fdiv_rn(m, 448.0f);
+    if (ok && blockIdx.x == 0) a.hdr[kHdrScaleS2] = __float_as_uint(s2);
+    *s_s2 = s2;
+    *s_ok = ok ? 1 : 0;
+  }
+  __syncthreads();
+  if (!*s_ok) return;
+  const float s2 = *s_s2;
+  const float4* h = static_cast<const float4*>(a.out);
+  uint32_t* q = static_cast<uint32_t*>(a.inter_q);
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < a.requant_n4;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldcg(h + i);
+    q[i] = pack_e4m3x4(__fdiv_rn(v.x, s2), __fdiv_rn(v.y, s2), __fdiv_rn(v.z, s2), __fdiv_rn(v.w, s2));
+  }
+}
+
 template <Orient O, Proj P, bool FP8, int KA, int BNT>
 __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_w,
@@ -230,6 +337,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(tmem_slot + 2);   // per epilogue warp amax (<= 8)
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
+  int* comb = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + 256 + C::kEpiBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -698,6 +806,47 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
+
+      if constexpr (!C::kDual) {
+        // ---- combine: a token's output tile is summed by the CTA that
+        // writes the last of its k slot pieces.  Every epilogue thread makes
+        // its slot rows visible (fence), then one thread per (token, tile)
+        // of the unit takes a ticket; the thread that draws k - 1 lists the
+        // pair, and the epilogue warps sum the listed pairs.  Integer tickets
+        // only; the sums run in slot order, so the result does not depend
+        // on which CTA finishes last.
+        if (a.tickets != nullptr) {
+          constexpr int kEpiThreads = 32 * C::kEpiWarps;
+          const int et = threadIdx.x - 64;          // 0 .. kEpiThreads - 1
+          int* list = comb + (it & 1) * (C::kCombList + 4);
+          int* nlist = list + C::kCombList;
+          if (et == 0) *nlist = 0;
+          __threadfence();
+          epilogue_bar<kEpiThreads>();
+          // swap-AB: one tile (the unit's 128 H rows), tokens n < nv;
+          // normal: two tiles (256 H columns), tokens r < nv
+          const int r = C::kSwap ? et : (et & (kTileM - 1));
+          const int tile = C::kSwap ? mt : 2 * mt + (et >> 7);
+          if (r < nv && (C::kSwap ? et < kTileM : true)) {
+            const int f = a.perm[p0 + r];
+            if (f >= 0 && f < a.num_assign) {
+              const int t = f / a.top_k;
+              const int ntile = a.ld_out / kTicketCols;
+              if (atom_add_acq_rel(a.tickets + static_cast<size_t>(t) * ntile + tile, 1) == a.top_k - 1)
+                list[atomicAdd(nlist, 1)] = t * 64 + tile;
+            }
+          }
+          epilogue_bar<kEpiThreads>();
+          const int n = *nlist;
+          if (n > 0) {
+            __threadfence();
+            for (int i = (warp - 2); i < n; i += C::kEpiWarps) {
+              const int v = list[i];
+              combine_tile(a, v >> 6, v & 63, lane);
+            }
+          }
+        }
+      }
     }
     if constexpr (FP8 && C::kDual) {
 #pragma unroll
@@ -718,6 +867,9 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     }
   }
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if constexpr (FP8 && C::kDual) {
+    if (a.amax_n > 0) requant_tail(a, red, abort_flag);   // red / abort_flag reused as smem words
+  }
 }
 
 template <Orient O, Proj P, bool FP8, int KA, int BNT>

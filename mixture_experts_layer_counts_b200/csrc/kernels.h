@@ -59,6 +59,7 @@ struct RouterArgs {
   uint32_t* hdr;
   float* rsplit;          // router_split_floats(T, E) floats, or NULL (no split-K)
   int invariant;          // 1: one logits kernel and summation order for every T (no split-K)
+  int* tickets;           // [T, H / kTicketCols] combine tickets, zeroed by the top-k kernel (may be NULL)
 };
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
 
@@ -90,13 +91,9 @@ cudaError_t launch_gather(const __nv_bfloat16* hidden, const int32_t* perm, int 
 cudaError_t launch_unpermute_rows(const void* src, const int32_t* inv_perm, int T, int k, int row_bytes,
                                   void* dst, cudaStream_t st);
 
-// FP8: s2 = max(amax_cta[0..n)) / 448, inter = E4M3(h32 / s2)
-cudaError_t launch_requant(const float* h32, const float* amax_cta, int n_cta, size_t count,
-                           uint32_t* hdr, uint8_t* inter, cudaStream_t st);
 
-// out[t, :] = bf16( sum_{j<k} ysc[t*k + j, :] ), j ascending
-cudaError_t launch_combine(const float* ysc, int T, int k, int H, __nv_bfloat16* out,
-                           cudaStream_t st);
+// out[t, :] = bf16( sum_{g < G} parts[g, t, :] ), g ascending (fp32 sum)
+cudaError_t launch_sum_partials(const float* parts, int G, long long n, __nv_bfloat16* out, cudaStream_t st);
 
 struct GemmArgs {
   const int4* chunks;          // {expert, first row in perm order, rows, index inside expert}
@@ -113,12 +110,20 @@ struct GemmArgs {
   int num_assign;              // T * top_k (bounds of perm values)
   const float* wscale;         // FP8 per-expert weight scale
   const uint32_t* act_scale;   // FP8: header word with s1 (w13) or s2 (w2)
-  float* amax_cta;             // FP8 w13: per-CTA amax|h|
+  float* amax_cta;             // FP8 w13: per-CTA amax|h| (this launch's slots)
+  const float* amax_all;       // FP8 w13, last launch of the call: every launch's per-CTA amax ...
+  int amax_n;                  // ... (amax_n slots); > 0 makes this launch requantise the whole
+  void* inter_q;               // intermediate into inter_q (E4M3) after a grid barrier
+  long long requant_n4;        // A * I / 4
   uint32_t* hdr;
   float* partials;             // kMaxSlots fp32 partial tiles (split units)
   int* flags;                  // kMaxSlots flags, zero at launch
   unsigned long long timeout_ns;   // limit of every bounded wait in the kernel
   int inject_stall;            // failure-path test: CTA 0 leaves one stage unfilled
+  int* tickets;                // w2: [T, H / kTicketCols] combine tickets (zero at launch)
+  void* y_out;                 // w2: out [T, H], written by the combine in the epilogue:
+  int y_fp32;                  //   bf16 (0), or the unrounded fp32 sum (1, tensor-parallel partials)
+  int top_k;
   int whole_units;             // 1: whole units dealt round-robin (no K splits) and, for
                                // swap-AB, MMA N fixed at the largest chunk: every output
                                // element then sees the same operations whatever the batch

@@ -187,3 +187,40 @@ def get_status(workspace, stream=None):
     info = C.c_uint32(0)
     code = _lib.lib().moe_get_status(_ptr(workspace), _stream(stream), C.byref(info))
     return int(code), int(info.value)
+
+
+def moe_forward_partial(hidden, router_w, router_bias, w13_shard, w2_shard, top_k, w13_scale=None,
+                        w2_scale=None, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """One tensor-parallel rank's share of the layer: fp32 [T, H], unrounded
+    (see moe_forward_partial in include/moe.h).  w13_shard [E, 2 I_g, H] holds
+    the rank's gate rows then its up rows, w2_shard [E, H, I_g] the matching
+    down-projection columns (shard_expert_weights builds both)."""
+    _need(hidden, torch.bfloat16, "hidden")
+    _need(router_w, torch.bfloat16, "router_w")
+    _need(w13_shard, (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), "w13_shard")
+    _need(w2_shard, (torch.bfloat16, torch.uint8, torch.float8_e4m3fn), "w2_shard")
+    T, H = hidden.shape
+    E = router_w.shape[0]
+    I_g = w13_shard.shape[1] // 2
+    dt = dtype_code(w13_shard)
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.float32, device=hidden.device)
+    _need(out, torch.float32, "out")
+    if workspace is None:
+        workspace = make_workspace(T, H, E, I_g, top_k, dt, hidden.device)
+    rc = _lib.lib().moe_forward_partial(
+        _ptr(hidden), _ptr(router_w), _ptr(router_bias), _ptr(w13_shard), _ptr(w2_shard), _ptr(w13_scale),
+        _ptr(w2_scale), T, H, E, I_g, top_k, dt, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    check(rc, "moe_forward_partial")
+    return out
+
+
+def sum_partials(partials, out=None, stream=None) -> torch.Tensor:
+    """bf16 [T, H] = sum over ranks g = 0, 1, ... of partials[g] (fp32 [G, T, H]),
+    added in rank order and rounded once."""
+    _need(partials, torch.float32, "partials")
+    G, T, H = partials.shape
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=partials.device)
+    check(_lib.lib().moe_sum_partials(_ptr(partials), G, T, H, _ptr(out), _stream(stream)), "moe_sum_partials")
+    return out
