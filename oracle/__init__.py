@@ -23,3 +23,4 @@ from .moe_ref import (  # noqa: F401
     router_logits,
     silu_mul,
 )
+from .rope_ref import inv_rope_fp8_ref, inv_rope_ref, per_head_fp8_ref  # noqa: F401
