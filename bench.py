@@ -541,6 +541,48 @@ def measure_workload(name, wl, args, rank, world, local, steps_exact=None):
     return res, cpu
 
 
+ROPE_SHAPE = dict(T=16384, n_heads=32, head_dim=128, max_pos=8192)
+
+
+def measure_inv_rope(local, steps=200):
+    """Device time of the fused inverse-RoPE + per-head FP8 kernel on a
+    prefill-sized call (inputs larger than L2, L2 flushed between steps).
+    Algorithmic bytes: x read (2 B / element), codes written (1 B / element),
+    one fp32 scale per head written, one table row pair read per token."""
+    from mixture_experts_layer_counts_b200 import layer
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    T, nH, D, P = (ROPE_SHAPE[k] for k in ("T", "n_heads", "head_dim", "max_pos"))
+    g = torch.Generator(device=dev).manual_seed(11)
+    x = torch.randn(T, nH, D, generator=g, device=dev).to(torch.bfloat16)
+    pos = torch.randint(0, P, (T,), generator=g, device=dev, dtype=torch.int32)
+    ang = torch.arange(P, device=dev, dtype=torch.float64)[:, None] * \
+        (10000.0 ** (-torch.arange(D // 2, device=dev, dtype=torch.float64) * 2.0 / D))[None, :]
+    ct, st = torch.cos(ang).float().contiguous(), torch.sin(ang).float().contiguous()
+    codes = torch.empty(T, nH, D, dtype=torch.uint8, device=dev)
+    scales = torch.empty(T, nH, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(5):
+        layer.inv_rope_fp8_quant(x, pos, ct, st, codes, scales)
+    ev = [new_events(2, stream) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        layer.inv_rope_fp8_quant(x, pos, ct, st, codes, scales)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    nbytes = T * nH * D * 3 + T * nH * 4 + T * D * 4 + T * 4
+    pk = peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"shape": dict(ROPE_SHAPE), "us": 1e3 * ms, "algorithmic_bytes": nbytes,
+            "roofline": {"kernel": "inv_rope_fp8_kernel", "bound": "hbm", "achieved": gbs, "peak": pk["hbm"],
+                         "unit": "GB/s", "frac": gbs / pk["hbm"], "peak_kind": pk["kind"]},
+            "tokens_per_s": T / (ms * 1e-3), "steps": steps}
+
+
 def run_ours(args, wl, rank, world, local):
     pk = peaks()
     head, cpu = measure_workload(args.workload, wl, args, rank, world, local, steps_exact=args.steps)
@@ -572,6 +614,7 @@ def run_ours(args, wl, rank, world, local):
         line[key] = head[key]
     if nested:
         line["workloads"] = nested
+        line["inv_rope_fp8"] = measure_inv_rope(local)
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if rank == 0:

@@ -198,6 +198,31 @@ moe_status_t moe_forward_partial(const void *hidden, const void *router_w, const
 
 moe_status_t moe_sum_partials(const float *partials, int G, int T, int H, void *out, void *stream);
 
+/* Fused inverse rotary position embedding + per-head FP8 quantisation, the
+ * kernel the pages name as the third MoE serving fix (a fused RoPE + FP8
+ * quantisation kernel, per head, whose token count must stay a runtime value:
+ * "AWS details MoE kernel fixes for SageMaker, upstreams them to vLLM", third
+ * fix; "AWS Unveils MoE Kernel Optimizations...", "Eliminating Triton JIT
+ * Recompilation").  Nothing here is specialised per T.
+ *   x         [T, n_heads, head_dim] bf16 (device), head vectors that carry RoPE
+ *   positions [T] int32 (device), the table row of each token
+ *   cos_tab, sin_tab [max_pos, head_dim / 2] fp32 (device), the rotary table
+ *   codes     [T, n_heads, head_dim] E4M3 (device), scales [T, n_heads] fp32 (device)
+ * For each token and head, element i < D/2 pairs with element i + D/2 and the
+ * pair turns by minus its angle (c = cos_tab[pos, i], s = sin_tab[pos, i]):
+ *   y[i] = x[i] c + x[i + D/2] s,   y[i + D/2] = x[i + D/2] c - x[i] s
+ * in fp32 with every product and every sum rounded (no fused multiply-add);
+ * then scale = fp32(max |y|) / 448 (1 when the head is all zeros) and codes =
+ * E4M3(fp32(y / scale)), round-to-nearest-even, saturating to +-448.  A
+ * position outside [0, max_pos) gives that token's heads codes 0 and scale 0.
+ * head_dim in {16, 32, 64, 128, 256, 512}; x, the tables and codes 16-byte
+ * aligned; positions and scales 4-byte aligned.  Errors: INVALID_ARG (NULL),
+ * UNSUPPORTED_SHAPE, MISALIGNED before any launch; MOE_ERR_CUDA if the
+ * launch fails.  Asynchronous on `stream`; needs no workspace. */
+moe_status_t moe_inv_rope_fp8_quant(const void *x, const int32_t *positions, const float *cos_tab,
+                                    const float *sin_tab, int T, int n_heads, int head_dim, int max_pos,
+                                    uint8_t *codes, float *scales, void *stream);
+
 /* Router only: topk_ids [T, top_k] int32 and topk_w [T, top_k] fp32 (device),
  * same definition as in moe_forward.  Uses the workspace of moe_forward's
  * shape (moe_workspace_size with the same T, H, E, top_k; any I >= 128). */

@@ -24,7 +24,8 @@ STATUS = {
 # every symbol include/moe.h declares
 EXPORTS = ("moe_workspace_size", "moe_workspace_init", "moe_forward", "moe_forward_hostio",
            "moe_route", "moe_align", "moe_get_status", "moe_status_string", "moe_route_static",
-           "moe_forward_batch_invariant", "moe_cache_stats", "moe_forward_partial", "moe_sum_partials")
+           "moe_forward_batch_invariant", "moe_cache_stats", "moe_forward_partial", "moe_sum_partials",
+           "moe_inv_rope_fp8_quant")
 
 
 class DebugOut(C.Structure):
@@ -69,6 +70,8 @@ def lib() -> C.CDLL:
         L.moe_forward_partial.argtypes = [vp] * 7 + [i] * 6 + [vp, vp, sz, vp]
         L.moe_sum_partials.restype = i
         L.moe_sum_partials.argtypes = [vp, i, i, i, vp, vp]
+        L.moe_inv_rope_fp8_quant.restype = i
+        L.moe_inv_rope_fp8_quant.argtypes = [vp] * 4 + [i] * 4 + [vp, vp, vp]
         L.moe_route.restype = i
         L.moe_route.argtypes = [vp, vp, vp, i, i, i, i, vp, vp, vp, sz, vp]
         L.moe_route_static.restype = i

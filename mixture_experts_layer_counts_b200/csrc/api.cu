@@ -562,6 +562,22 @@ moe_status_t moe_sum_partials(const float* partials, int G, int T, int H, void* 
                                          static_cast<__nv_bfloat16*>(out), static_cast<cudaStream_t>(stream)));
 }
 
+moe_status_t moe_inv_rope_fp8_quant(const void* x, const int32_t* positions, const float* cos_tab,
+                                    const float* sin_tab, int T, int n_heads, int head_dim, int max_pos,
+                                    uint8_t* codes, float* scales, void* stream) {
+  if (!x || !positions || !cos_tab || !sin_tab || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  if (T < 1 || n_heads < 1 || max_pos < 1) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (head_dim != 16 && head_dim != 32 && head_dim != 64 && head_dim != 128 && head_dim != 256 &&
+      head_dim != 512)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(T) * n_heads * head_dim >= (1LL << 40)) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(x) || !aligned16(cos_tab) || !aligned16(sin_tab) || !aligned16(codes) ||
+      (reinterpret_cast<uintptr_t>(scales) & 3u) || (reinterpret_cast<uintptr_t>(positions) & 3u))
+    return MOE_ERR_MISALIGNED;
+  return cuda_status(launch_inv_rope_fp8(x, positions, cos_tab, sin_tab, T, n_heads, head_dim, max_pos, codes,
+                                         scales, static_cast<cudaStream_t>(stream)));
+}
+
 moe_status_t moe_route(const void* hidden, const void* router_w, const float* router_bias, int T,
                        int H, int E, int top_k, int32_t* topk_ids, float* topk_w, void* workspace,
                        size_t workspace_bytes, void* stream) {

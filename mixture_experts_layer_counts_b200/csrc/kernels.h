@@ -92,6 +92,11 @@ cudaError_t launch_unpermute_rows(const void* src, const int32_t* inv_perm, int 
                                   void* dst, cudaStream_t st);
 
 
+// Inverse RoPE + per-head E4M3 quantisation (rope.cu); D in {16, 32, 64, 128, 256, 512}
+cudaError_t launch_inv_rope_fp8(const void* x, const int32_t* pos, const float* cos_tab, const float* sin_tab,
+                                int T, int nH, int D, int max_pos, uint8_t* codes, float* scales,
+                                cudaStream_t st);
+
 // out[t, :] = bf16( sum_{g < G} parts[g, t, :] ), g ascending (fp32 sum)
 cudaError_t launch_sum_partials(const float* parts, int G, long long n, __nv_bfloat16* out, cudaStream_t st);
 

@@ -224,3 +224,22 @@ def sum_partials(partials, out=None, stream=None) -> torch.Tensor:
         out = torch.empty((T, H), dtype=torch.bfloat16, device=partials.device)
     check(_lib.lib().moe_sum_partials(_ptr(partials), G, T, H, _ptr(out), _stream(stream)), "moe_sum_partials")
     return out
+
+
+def inv_rope_fp8_quant(x, positions, cos_tab, sin_tab, codes=None, scales=None, stream=None):
+    """(codes [T, nH, D] uint8 E4M3, scales [T, nH] fp32) of the fused inverse
+    RoPE + per-head FP8 quantisation (see include/moe.h).  x [T, nH, D] bf16,
+    positions [T] int32, cos_tab / sin_tab [max_pos, D/2] fp32."""
+    _need(x, torch.bfloat16, "x")
+    _need(positions, torch.int32, "positions")
+    _need(cos_tab, torch.float32, "cos_tab")
+    _need(sin_tab, torch.float32, "sin_tab")
+    T, nH, D = x.shape
+    if codes is None:
+        codes = torch.empty((T, nH, D), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((T, nH), dtype=torch.float32, device=x.device)
+    check(_lib.lib().moe_inv_rope_fp8_quant(_ptr(x), _ptr(positions), _ptr(cos_tab), _ptr(sin_tab), T, nH, D,
+                                            cos_tab.shape[0], _ptr(codes), _ptr(scales), _stream(stream)),
+          "moe_inv_rope_fp8_quant")
+    return codes, scales

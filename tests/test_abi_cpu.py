@@ -76,3 +76,13 @@ def test_argument_errors_before_any_launch(L):
     assert L.moe_workspace_init(None, 0, None) == 1
     assert L.moe_align(None, 4, 8, 2, None, None, None, None, None, 0, None) == 1
     assert L.moe_align(C.c_void_p(16), 4, 2000, 2, None, None, None, None, None, 0, None) == 2
+
+
+def test_inv_rope_argument_errors(L):
+    p = C.c_void_p
+    f = L.moe_inv_rope_fp8_quant
+    assert f(None, p(16), p(16), p(16), 4, 2, 128, 10, p(16), p(16), None) == 1      # NULL x
+    assert f(p(16), p(16), p(16), p(16), 4, 2, 96, 10, p(16), p(16), None) == 2      # head_dim 96
+    assert f(p(16), p(16), p(16), p(16), 0, 2, 128, 10, p(16), p(16), None) == 2     # T = 0
+    assert f(p(24), p(16), p(16), p(16), 4, 2, 128, 10, p(16), p(16), None) == 7     # x not 16-byte aligned
+    assert f(p(16), p(16), p(16), p(16), 4, 2, 128, 10, p(16), p(18), None) == 7     # scales not 4-byte aligned
