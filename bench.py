@@ -297,11 +297,13 @@ SWAP_MAX_TOKENS = 64   # the library's default swap-AB / normal threshold (token
 def launches_per_step(wl, T):
     """Kernels one layer call launches: router (logits, top-k), align (two
     slice grids from T*k = 8192 on), gather, w13 and w2 GEMMs (one per
-    orientation in use; the FP8 requantisation closes the last w13 launch and
-    the combine runs in the w2 epilogue)."""
+    orientation in use; the FP8 requantisation closes the last w13 launch),
+    and the combine pass when normal-orientation experts are present (else
+    the w2 epilogue combines)."""
     any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
     n_align = 2 if T * wl["top_k"] >= 8192 else 1
-    return 2 + n_align + 1 + 2 * (2 if any_normal else 1)
+    # with normal-orientation experts the combine is a separate pass
+    return 2 + n_align + 1 + 2 * (2 if any_normal else 1) + (1 if any_normal else 0)
 
 
 def new_events(n, stream):

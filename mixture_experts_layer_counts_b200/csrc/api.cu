@@ -285,7 +285,11 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g2.amax_cta = nullptr;
   g2.amax_n = 0;
   g2.inject_stall = 0;
-  g2.tickets = at<int>(ws, L.tickets);   // zeroed by the router's top-k kernel
+  // Combine: when every expert runs swap-AB (decode batches) the down GEMM's
+  // epilogue combines (tickets); with normal-orientation experts the slot rows
+  // are summed by a separate pass (the epilogue's combine reads would then
+  // compete with the tensor-bound mainloop; measured slower)
+  g2.tickets = any_normal ? nullptr : at<int>(ws, L.tickets);   // zeroed by the router's top-k kernel
   g2.y_out = out;
   g2.y_fp32 = out_fp32 ? 1 : 0;
   g2.top_k = k;
@@ -305,7 +309,9 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.flags = flags + 3 * kMaxSlots;
     MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
   }
-  record(dbg, 6, st);   // the combine runs inside the down-projection GEMM's epilogue
+  record(dbg, 6, st);
+  if (any_normal)
+    MOE_TRY(cuda_status(launch_combine(at<float>(ws, L.ysc), T, k, H, out, out_fp32, st)));
   record(dbg, 7, st);
 
   if (dbg) {

@@ -2,6 +2,9 @@
 //   gather   x_perm[p] = hidden[perm[p] / k]  (bf16), or its per-tensor E4M3
 //            quantisation x / s1 (FP8 path; one IEEE fp32 division, RNE,
 //            saturating to +-448)
+//   combine  out[t] = bf16(sum_{j<k} ysc[t*k + j]) in slot order, fp32 sum
+//            (calls with normal-orientation experts; otherwise the down GEMM's
+//            epilogue combines)
 // All grids are sized from the SM count; 16-byte vector accesses.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -86,6 +89,61 @@ __global__ void gather_quant_kernel(const uint4* __restrict__ hidden, const int3
     }
     xq[i] = make_uint2(pack_e4m3x4(f[0], f[1], f[2], f[3]), pack_e4m3x4(f[4], f[5], f[6], f[7]));
   }
+}
+
+// Combine pass (used when some experts run in the normal orientation):
+// out[t] = sum_{j<k} ysc[t*k + j] in slot order, fp32, then one bf16 rounding
+// (or the unrounded fp32 sum for a tensor-parallel partial).  Work unit =
+// (token t, block of 256 float4 columns); per thread the k slot loads are
+// issued together and summed in slot order.
+__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ ysc, int T, int k,
+                                                      int h4, void* __restrict__ out, int out_f32) {
+  pdl_wait();
+  pdl_launch_next();
+  const int nb = (h4 + 255) / 256;
+  const int units = T * nb;
+  for (int unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    const int t = unit / nb;
+    const int c = (unit - t * nb) * 256 + threadIdx.x;
+    if (c >= h4) continue;
+    const float4* src = ysc + static_cast<size_t>(t) * k * h4 + c;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j0 = 0; j0 < k; j0 += 8) {
+      float4 y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (j0 + u < k) y[u] = __ldcg(src + static_cast<size_t>(j0 + u) * h4);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u < k) {
+          if (j0 + u == 0) {
+            acc = y[u];
+          } else {
+            acc.x += y[u].x;
+            acc.y += y[u].y;
+            acc.z += y[u].z;
+            acc.w += y[u].w;
+          }
+        }
+      }
+    }
+    if (out_f32) {
+      static_cast<float4*>(out)[static_cast<size_t>(t) * h4 + c] = acc;
+    } else {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      static_cast<uint2*>(out)[static_cast<size_t>(t) * h4 + c] =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
+  }
+}
+
+cudaError_t launch_combine(const float* ysc, int T, int k, int H, void* out, bool out_f32, cudaStream_t st) {
+  const int h4 = H / 4;
+  const int units = T * ((h4 + 255) / 256);
+  const int grid = std::min(units, sm_count() * 8);
+  return launch_pdl(combine_kernel, dim3(grid), dim3(256), 0, st, reinterpret_cast<const float4*>(ysc), T, k,
+                    h4, out, out_f32 ? 1 : 0);
 }
 
 // Tensor-parallel sum: out[i] = bf16(parts[0][i] + parts[1][i] + ... ), the

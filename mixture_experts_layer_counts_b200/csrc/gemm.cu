@@ -25,11 +25,13 @@
 //          grid barrier and the per-tensor E4M3 requantisation of h
 //          (requant_tail), so no separate pass is launched.
 //   kW2  : one accumulator; the epilogue multiplies by the router weight
-//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), then
+//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot).  When
+//          every expert of the call runs swap-AB (decode batches), it then
 //          takes an integer ticket per (token, 128-column tile); the CTA that
 //          writes a token's last slot of a tile sums the k slot rows in slot
-//          order and writes the bf16 output (combine_tile): the combine runs
-//          inside this kernel, deterministic, no floating-point atomics.
+//          order and writes the output (combine_tile), so the combine runs
+//          inside this kernel; otherwise a separate pass sums the slot rows in
+//          the same order.  Deterministic, no floating-point atomics.
 //
 // Work split.  A "unit" is one output tile (token chunk x weight-row tile)
 // and needs `katoms` K atoms.
@@ -310,10 +312,19 @@ __device__ __forceinline__ void requant_tail(const GemmArgs& a, float* s_s2, vol
   const float s2 = *s_s2;
   const float4* h = static_cast<const float4*>(a.out);
   uint32_t* q = static_cast<uint32_t*>(a.inter_q);
-  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < a.requant_n4;
-       i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const float4 v = __ldcg(h + i);
-    q[i] = pack_e4m3x4(__fdiv_rn(v.x, s2), __fdiv_rn(v.y, s2), __fdiv_rn(v.z, s2), __fdiv_rn(v.w, s2));
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  constexpr int kU = 8;   // loads in flight per thread
+  for (long long i0 = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i0 < a.requant_n4;
+       i0 += kU * stride) {
+    float4 v[kU];
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (i0 + u * stride < a.requant_n4) v[u] = __ldcg(h + i0 + u * stride);
+#pragma unroll
+    for (int u = 0; u < kU; ++u)
+      if (i0 + u * stride < a.requant_n4)
+        q[i0 + u * stride] = pack_e4m3x4(__fdiv_rn(v[u].x, s2), __fdiv_rn(v[u].y, s2), __fdiv_rn(v[u].z, s2),
+                                         __fdiv_rn(v[u].w, s2));
   }
 }
 
@@ -809,19 +820,21 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
 
       if constexpr (!C::kDual) {
         // ---- combine: a token's output tile is summed by the CTA that
-        // writes the last of its k slot pieces.  Every epilogue thread makes
-        // its slot rows visible (fence), then one thread per (token, tile)
-        // of the unit takes a ticket; the thread that draws k - 1 lists the
-        // pair, and the epilogue warps sum the listed pairs.  Integer tickets
-        // only; the sums run in slot order, so the result does not depend
-        // on which CTA finishes last.
+        // writes the last of its k slot pieces.  After a barrier of the
+        // epilogue warps (every slot row of the unit stored), one thread per
+        // (token, tile) of the unit takes a ticket with release/acquire
+        // semantics; the thread that draws k - 1 lists the pair, and the
+        // epilogue warps sum the listed pairs, reading through L2.  Integer
+        // tickets only; the sums run in slot order, so the result does not
+        // depend on which CTA finishes last.
         if (a.tickets != nullptr) {
           constexpr int kEpiThreads = 32 * C::kEpiWarps;
           const int et = threadIdx.x - 64;          // 0 .. kEpiThreads - 1
           int* list = comb + (it & 1) * (C::kCombList + 4);
           int* nlist = list + C::kCombList;
           if (et == 0) *nlist = 0;
-          __threadfence();
+          // every epilogue thread's slot-row stores precede the barrier; the
+          // ticket's release (acq_rel at GPU scope) publishes them with it
           epilogue_bar<kEpiThreads>();
           // swap-AB: one tile (the unit's 128 H rows), tokens n < nv;
           // normal: two tiles (256 H columns), tokens r < nv
@@ -839,7 +852,6 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
           epilogue_bar<kEpiThreads>();
           const int n = *nlist;
           if (n > 0) {
-            __threadfence();
             for (int i = (warp - 2); i < n; i += C::kEpiWarps) {
               const int v = list[i];
               combine_tile(a, v >> 6, v & 63, lane);

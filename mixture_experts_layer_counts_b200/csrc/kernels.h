@@ -97,6 +97,9 @@ cudaError_t launch_inv_rope_fp8(const void* x, const int32_t* pos, const float* 
                                 int T, int nH, int D, int max_pos, uint8_t* codes, float* scales,
                                 cudaStream_t st);
 
+// out[t, :] = bf16( sum_{j<k} ysc[t*k + j, :] ), j ascending (fp32 sum), or the fp32 sum
+cudaError_t launch_combine(const float* ysc, int T, int k, int H, void* out, bool out_f32, cudaStream_t st);
+
 // out[t, :] = bf16( sum_{g < G} parts[g, t, :] ), g ascending (fp32 sum)
 cudaError_t launch_sum_partials(const float* parts, int G, long long n, __nv_bfloat16* out, cudaStream_t st);
 

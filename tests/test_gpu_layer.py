@@ -8,8 +8,9 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import (WEIGHT_ATOL, assert_fp8_scales_and_codes, assert_inter_equal, assert_output_close,
-                     assert_routing_equal, bf16_rounding_ambiguity, custom_inputs, oracle_of)
+from helpers import (PARITY_LOG, WEIGHT_ATOL, assert_fp8_scales_and_codes, assert_inter_equal,
+                     assert_output_close, assert_routing_equal, bf16_rounding_ambiguity, custom_inputs,
+                     oracle_of)
 from mixture_experts_layer_counts_b200 import layer
 from mixture_experts_layer_counts_b200.inputs import (WORKLOADS, host_bits, make_hidden, make_inputs,
                                                       make_router, zipf_bias)
@@ -302,7 +303,15 @@ def test_forward_prefill_sampled(cuda_ok):
     tokens = np.sort(np.concatenate([[0, 4095], rng.choice(np.arange(1, 4095), 254, replace=False)]))
     ref = oracle_of(inp, tokens=tokens)
     assert_routing_equal(dbg, ref)                    # routing of all 4096 tokens
-    assert_output_close(out, ref, fp8=False, tokens=tokens)
+    # About 1e-4 of the intermediate values have an exact h within the fp32
+    # error of a bf16 rounding boundary, so the GPU may round them to the other
+    # neighbour (a correct result); over a million outputs a few near-zero
+    # elements can then move by more than the bound's absolute term.  Those
+    # elements must be explained by the envelope, and stay rare.
+    _, env = bf16_rounding_ambiguity(inp, ref, tokens=tokens)
+    assert_output_close(out, ref, fp8=False, tokens=tokens, env=env)
+    rec = PARITY_LOG[-1]
+    assert rec["n_over_strict"] <= 1e-5 * out[tokens].numel(), rec
 
 
 def test_deterministic(cuda_ok):
