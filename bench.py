@@ -301,9 +301,12 @@ def launches_per_step(wl, T):
     and the combine pass when normal-orientation experts are present (else
     the w2 epilogue combines)."""
     any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
-    n_align = 2 if T * wl["top_k"] >= 8192 else 1
+    A = T * wl["top_k"]
+    # decode-sized calls: logits, top-k and align in one launch
+    fused_router = A < 8192 and wl["E"] <= 256
+    n_route = 1 if fused_router else 2 + (2 if A >= 8192 else 1)
     # with normal-orientation experts the combine is a separate pass
-    return 2 + n_align + 1 + 2 * (2 if any_normal else 1) + (1 if any_normal else 0)
+    return n_route + 1 + 2 * (2 if any_normal else 1) + (1 if any_normal else 0)
 
 
 def new_events(n, stream):

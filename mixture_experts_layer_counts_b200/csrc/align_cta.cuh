@@ -99,7 +99,7 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int f = base + 32 * u + lane;
-      ev[u] = f < end ? a.topk_ids[f] : -1;
+      ev[u] = f < end ? __ldcg(a.topk_ids + f) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -160,7 +160,7 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int f = base + 32 * u + lane;
-      ev[u] = f < end ? a.topk_ids[f] : -1;
+      ev[u] = f < end ? __ldcg(a.topk_ids + f) : -1;
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {

@@ -211,9 +211,12 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                at<int4>(ws, L.chunks_pair),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
                at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots, at<int>(ws, L.slice_hist)};
-  MOE_TRY(cuda_status(launch_router(ra, st)));
+  // Decode-sized calls run logits, top-k and align in one launch (the
+  // "router" stage then covers the align too and the "align" stage is empty).
+  bool fused_route = false;
+  MOE_TRY(cuda_status(launch_router(ra, st, invariant ? nullptr : &aa, &fused_route)));
   record(dbg, 1, st);
-  MOE_TRY(cuda_status(launch_align(aa, st)));
+  if (!fused_route) MOE_TRY(cuda_status(launch_align(aa, st)));
   record(dbg, 2, st);
 
   MOE_TRY(cuda_status(launch_gather(static_cast<const __nv_bfloat16*>(hidden), at<int32_t>(ws, L.perm),

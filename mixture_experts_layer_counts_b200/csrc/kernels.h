@@ -61,7 +61,11 @@ struct RouterArgs {
   int invariant;          // 1: one logits kernel and summation order for every T (no split-K)
   int* tickets;           // [T, H / kTicketCols] combine tickets, zeroed by the top-k kernel (may be NULL)
 };
-cudaError_t launch_router(const RouterArgs& a, cudaStream_t st);
+struct AlignArgs;
+// fuse_align non-NULL: a decode-sized call may run logits, top-k and align in
+// one launch (then *fused is set and the align must not be launched again).
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align = nullptr,
+                          bool* fused = nullptr);
 
 struct AlignArgs {
   const int32_t* topk_ids;

@@ -47,7 +47,7 @@ StaticRouteLayout static_route_layout(int T, int E) {
     off = align_up(off + bytes, 1024);
     return o;
   };
-  L.header = take(kHeaderBytes);
+  L.header = take(kStatusBytes);
   L.logits = take(static_cast<size_t>(T) * E * 4);
   L.xnorm = take(static_cast<size_t>(T) * 4);
   L.wnorm = take(static_cast<size_t>(E) * 4);
@@ -96,7 +96,7 @@ extern "C" moe_status_t moe_route_static(const void* hidden, const void* router_
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // only the header (status / counters) must start at zero; every other
   // region is written before it is read within the call
-  if (cudaMemsetAsync(b + L.header, 0, kHeaderBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemsetAsync(b + L.header, 0, kStatusBytes, st) != cudaSuccess) return MOE_ERR_CUDA;
   RouterArgs ra{static_cast<const __nv_bfloat16*>(hidden), static_cast<const __nv_bfloat16*>(router_w),
                 router_bias, T, H, E, top_k,
                 reinterpret_cast<float*>(b + L.logits), reinterpret_cast<float*>(b + L.xnorm),

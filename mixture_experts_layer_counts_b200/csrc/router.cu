@@ -21,6 +21,7 @@
 
 #include <cfloat>
 
+#include "align_cta.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -193,7 +194,8 @@ template <int TT, int ACC>
 __device__ __forceinline__ void logits_body(
     const __nv_bfloat16* __restrict__ hidden, const __nv_bfloat16* __restrict__ router_w,
     const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits,
-    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok, uint4* sx) {
+    float* __restrict__ xnorm, float* __restrict__ wnorm, float* __restrict__ amax_tok, uint4* sx,
+    bool every_cta_wnorm = false) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = blockDim.x >> 5;
   const int t0 = blockIdx.x * TT;
@@ -306,7 +308,7 @@ __device__ __forceinline__ void logits_body(
     const float b = bias ? bias[e] : 0.f;
     for (int tt = 0; tt < nt; ++tt)
       logits[static_cast<size_t>(t0 + tt) * E + e] = static_cast<float>(acc[tt] + static_cast<Acc>(b));
-    if (blockIdx.x == 0) wnorm[e] = sqrtf(wsq);
+    if (blockIdx.x == 0 || every_cta_wnorm) wnorm[e] = sqrtf(wsq);
   }
 }
 
@@ -746,6 +748,80 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Fused decode router: logits, top-k and align in one launch, without
+// serialising the top-k of all tokens on one SM.  CTA (token tile, expert
+// group) computes its logits (every CTA also writes ||w_e|| of its experts,
+// identical values, so a token tile needs no other tile's CTAs); after a
+// barrier its thread 0 takes a ticket of the token tile (acquire-release at
+// GPU scope); the CTA that completes the tile runs the top-k of the tile's
+// tokens (one warp per token), then takes a ticket of the whole grid; the CTA
+// that completes the grid runs the align (the one-CTA form).  Tickets only:
+// no CTA ever waits for another, and each counter is reset by the CTA that
+// completes it, so every call starts from zero.  Used for decode-sized calls
+// (T*k < kAlignSliceMin, E <= 256, token tiles <= kRouterFusedMaxTiles).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned int ticket_acq_rel(uint32_t* p) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
+
+template <int TT, int ACC, int kPer>
+__global__ void __launch_bounds__(256) router_fused_kernel(RouterArgs ra, AlignArgs aa, float gamma,
+                                                           float ulast) {
+  extern __shared__ uint4 sx[];
+  __shared__ int s_last;
+  pdl_wait();
+  pdl_launch_next();
+  logits_body<TT, ACC>(ra.hidden, ra.router_w, ra.bias, ra.T, ra.H, ra.E, ra.logits, ra.xnorm, ra.wnorm,
+                       ra.amax_tok, sx, true);
+  __syncthreads();   // every logit, norm and amax of this CTA is stored
+  if (threadIdx.x == 0) {
+    uint32_t* cnt = ra.hdr + kHdrRouterTiles + blockIdx.x;
+    const bool last = ticket_acq_rel(cnt) == gridDim.y - 1;
+    if (last) *cnt = 0u;
+    s_last = last ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  // this CTA completes token tile blockIdx.x: top-k of its tokens
+  const int t0 = blockIdx.x * TT;
+  const int nt = min(TT, ra.T - t0);
+  for (int tt = threadIdx.x >> 5; tt < nt; tt += blockDim.x >> 5) {
+    const int t = t0 + tt;
+    if (ra.tickets != nullptr)
+      for (int i = threadIdx.x & 31; i < ra.H / kTicketCols; i += 32)
+        ra.tickets[static_cast<size_t>(t) * (ra.H / kTicketCols) + i] = 0;
+    topk_token<kPer>(t, ra.logits, ra.xnorm, ra.wnorm, ra.amax_tok, ra.rsplit, 1, ra.bias, ra.hidden,
+                     ra.router_w, ra.T, ra.H, ra.E, ra.k, gamma, ulast, ra.topk_ids, ra.topk_w, ra.cand, ra.hdr);
+  }
+  __syncthreads();   // every top-k of the tile is stored
+  if (threadIdx.x == 0) {
+    uint32_t* cnt = ra.hdr + kHdrRouterAll;
+    const bool last = ticket_acq_rel(cnt) == gridDim.x - 1;
+    if (last) *cnt = 0u;
+    s_last = last ? 1 : 0;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  // this CTA completes the grid: the align, in the one-CTA form (the dynamic
+  // shared memory holds its per-warp histograms)
+  align_cta(aa, 0, 0, reinterpret_cast<int*>(sx));
+}
+
+template <int TT, int ACC, int kPer>
+static cudaError_t launch_fused(const RouterArgs& a, const AlignArgs& aa, float gamma, float ulast,
+                                cudaStream_t st) {
+  auto kern = router_fused_kernel<TT, ACC, kPer>;
+  const int hist = 8 * a.E * 4;
+  const int smem = TT * a.H * 2 > hist ? TT * a.H * 2 : hist;
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((a.T + TT - 1) / TT, (a.E + 7) / 8);
+  return launch_pdl(kern, grid, dim3(256), smem, st, a, aa, gamma, ulast);
+}
+
+// ---------------------------------------------------------------------------
 template <int TT, int ACC>
 static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
   auto kern = router_logits_kernel<TT, ACC>;
@@ -847,7 +923,8 @@ static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStre
                     a.logits, a.xnorm, a.wnorm, a.amax_tok, a.rsplit);
 }
 
-cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align, bool* fused) {
+  if (fused) *fused = false;
   // fp64 accumulation while the logit work is small (decode batches); fp32
   // with the wider certified bound for large batches
   // fp64 accumulation while the logit work is small (decode batches): per
@@ -891,6 +968,35 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
         break;
       }
     }
+    // decode-sized calls: logits, top-k and align in one launch
+    const long long A = static_cast<long long>(a.T) * a.k;
+    const int tiles = (a.T + tt - 1) / tt;
+    if (fuse_align != nullptr && fused != nullptr && mode != kAcc32 && tt <= 4 && a.E <= 256 &&
+        A < kAlignSliceMin && tiles <= kRouterFusedMaxTiles && a.rsplit != nullptr) {
+      const int nchain_f = a.H / 32 + 16;
+      const double u32f = 5.9604644775390625e-08, u64f = 1.1102230246251565e-16;
+      const float gamma_f = mode == kAcc64 ? static_cast<float>(nchain_f * u64f * 1.0001)
+                                           : static_cast<float>((7.0 * u32f + nchain_f * u64f) * 1.0001);
+      const float ulast_f = static_cast<float>(u32f);
+      const int ecls = a.E <= 64 ? 0 : (a.E <= 128 ? 1 : 2);   // experts per lane 2, 4, 8
+      const int ti = tt == 1 ? 0 : (tt == 2 ? 1 : 2);
+      cudaError_t e2;
+      switch ((mode == kAcc64 ? 0 : 9) + 3 * ecls + ti) {
+#define MOE_FUSED_CASE(I, TT_, ACC_, KP_) \
+  case I: e2 = launch_fused<TT_, ACC_, KP_>(a, *fuse_align, gamma_f, ulast_f, st); break;
+        MOE_FUSED_CASE(0, 1, kAcc64, 2) MOE_FUSED_CASE(1, 2, kAcc64, 2) MOE_FUSED_CASE(2, 4, kAcc64, 2)
+        MOE_FUSED_CASE(3, 1, kAcc64, 4) MOE_FUSED_CASE(4, 2, kAcc64, 4) MOE_FUSED_CASE(5, 4, kAcc64, 4)
+        MOE_FUSED_CASE(6, 1, kAcc64, 8) MOE_FUSED_CASE(7, 2, kAcc64, 8) MOE_FUSED_CASE(8, 4, kAcc64, 8)
+        MOE_FUSED_CASE(9, 1, kAccMixed, 2) MOE_FUSED_CASE(10, 2, kAccMixed, 2) MOE_FUSED_CASE(11, 4, kAccMixed, 2)
+        MOE_FUSED_CASE(12, 1, kAccMixed, 4) MOE_FUSED_CASE(13, 2, kAccMixed, 4)
+        MOE_FUSED_CASE(14, 4, kAccMixed, 4) MOE_FUSED_CASE(15, 1, kAccMixed, 8)
+        MOE_FUSED_CASE(16, 2, kAccMixed, 8)
+        default: e2 = launch_fused<4, kAccMixed, 8>(a, *fuse_align, gamma_f, ulast_f, st); break;
+#undef MOE_FUSED_CASE
+      }
+      if (e2 == cudaSuccess) *fused = true;
+      return e2;
+    }
     switch (mode * 32 + tt) {
       case kAcc64 * 32 + 16: err = launch_logits<16, kAcc64>(a, st); break;
       case kAcc64 * 32 + 8: err = launch_logits<8, kAcc64>(a, st); break;
@@ -920,6 +1026,7 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st) {
                                           : static_cast<float>(nchain * u32 * 1.0001);
   const float ulast = mode != kAcc32 ? static_cast<float>(u32) : static_cast<float>(2.0 * u32);
   if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, nsplit, st);
+  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, nsplit, st);
   if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, nsplit, st);
   return launch_topk<kMaxExperts / 32>(a, gamma, ulast, nsplit, st);
 }
