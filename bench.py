@@ -503,6 +503,14 @@ def measure_workload(name, wl, args, rank, world, local, steps_exact=None):
         layer_frac = {"layer_tflops_frac_of_burst": flops / (ms_per_step * 1e-3) / 1e12 / (mult * pk["bf16"]),
                       "layer_tflops_frac_of_sustained":
                           flops / (ms_per_step * 1e-3) / 1e12 / (mult * pk["bf16_sustained"])}
+    elif dt == 0 and T <= 32 and not args.batch_invariant and os.environ.get("MOE_FUSED_FFN", "1") != "0":
+        # bf16 decode batches: gate/up and down GEMMs are one launch (ffn_swap_kernel);
+        # the bracket covers it, its bytes are every activated weight byte
+        achieved = weight_bytes / w13_s / 1e9
+        roof = {"kernel": "ffn_swap_kernel (gate/up + down GEMMs, one launch)", "bound": "hbm",
+                "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s", "frac": achieved / pk["hbm"],
+                "peak_kind": pk["kind"], "algorithmic_bytes_per_launch": weight_bytes}
+        layer_frac = {}
     else:
         achieved = w13_bytes / w13_s / 1e9
         roof = {"kernel": "grouped_gemm_kernel<swap-AB, w13>", "bound": "hbm", "achieved": achieved,

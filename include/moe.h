@@ -95,7 +95,9 @@ typedef struct {
   void **stage_events; /* host array of 8 cudaEvent_t recorded on `stream` at the stage
                           boundaries: start, router, align, gather, w13, requant, w2, combine */
   int force_orient;    /* 0 = per-expert choice, 1 = swap-AB for all experts,
-                          2 = normal orientation for all experts (testing) */
+                          2 = normal orientation for all experts, 3 = swap-AB for all
+                          experts with one launch per GEMM (no fused decode FFN)
+                          (testing) */
   int wait_timeout_us; /* limit of each bounded device-side wait (0 = 2 s) */
   int inject_stall;    /* failure-path test: 1 makes the first gate/up GEMM CTA leave one
                           pipeline stage unfilled, so a bounded wait expires and the call

@@ -100,6 +100,17 @@ int swap_threshold() {
   return v;
 }
 
+// The fused decode FFN launch is on by default; MOE_FUSED_FFN=0 selects the
+// two-launch path (for measurements).
+bool fused_ffn_enabled() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = std::getenv("MOE_FUSED_FFN");
+    v = (s && std::atoi(s) == 0) ? 0 : 1;
+  }
+  return v == 1;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 moe_status_t check_shape(int T, int H, int E, int I, int k, int dtype) {
@@ -172,7 +183,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   uint32_t* hdr = at<uint32_t>(ws, L.header);
 
   int tau = swap_threshold();
-  if (dbg && dbg->force_orient == 1) tau = INT_MAX;
+  if (dbg && (dbg->force_orient == 1 || dbg->force_orient == 3)) tau = INT_MAX;
   if (dbg && dbg->force_orient == 2) tau = 0;
   if (H % 256 != 0) tau = INT_MAX;   // the normal-orientation w2 tile is 256 rows of H
   if (invariant) tau = INT_MAX;       // one orientation for every expert and batch
@@ -210,7 +221,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
                at<int4>(ws, L.chunks_pair),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
-               at<int>(ws, L.gemm_flags), kGemmLaunches * kMaxSlots, at<int>(ws, L.slice_hist)};
+               at<int>(ws, L.gemm_flags), L.n_gemm_flags, at<int>(ws, L.slice_hist)};
   // Decode-sized calls run logits, top-k and align in one launch (the
   // "router" stage then covers the align too and the "align" stage is empty).
   bool fused_route = false;
@@ -254,29 +265,6 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     g.inter_q = inter;
     g.requant_n4 = static_cast<long long>(A) * I / 4;
   };
-  if (any_swap) {
-    GemmArgs g = g13;
-    g.chunks = at<int4>(ws, L.chunks_swap);
-    g.nchunks = hdr + kHdrChunksSwap;
-    g.mtiles = I / kTileM;
-    g.amax_cta = amax_cta;
-    g.flags = flags + 0 * kMaxSlots;
-    requant_args(g, !any_normal);
-    MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW13, fp8, tw13s, txs, g, grid, st)));
-  }
-  if (any_normal) {
-    GemmArgs g = g13;
-    g.chunks = at<int4>(ws, L.chunks_pair);
-    g.nchunks = hdr + kHdrChunksPair;
-    g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
-    g.amax_cta = amax_cta + (any_swap ? grid : 0);
-    g.flags = flags + 1 * kMaxSlots;
-    requant_args(g, true);
-    MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
-  }
-  record(dbg, 4, st);   // (the FP8 requantisation ran at the end of the gate/up GEMM)
-  record(dbg, 5, st);
-
   GemmArgs g2 = g13;
   g2.katoms = I * (fp8 ? 1 : 2) / kAtomBytes;
   g2.w_rows_per_expert = H;
@@ -296,21 +284,66 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g2.y_out = out;
   g2.y_fp32 = out_fp32 ? 1 : 0;
   g2.top_k = k;
-  if (any_swap) {
-    GemmArgs g = g2;
-    g.chunks = at<int4>(ws, L.chunks_swap);
-    g.nchunks = hdr + kHdrChunksSwap;
-    g.mtiles = H / kTileM;
-    g.flags = flags + 2 * kMaxSlots;
-    MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, fp8, tw2s, tis, g, grid, st)));
-  }
-  if (any_normal) {
-    GemmArgs g = g2;
-    g.chunks = at<int4>(ws, L.chunks_normal);
-    g.nchunks = hdr + kHdrChunksNormal;
-    g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
-    g.flags = flags + 3 * kMaxSlots;
-    MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
+  // Decode batches in bf16 (T <= 32, every expert swap-AB): both GEMMs in one
+  // persistent launch (ffn.cu); otherwise one launch per GEMM and orientation.
+  const bool use_ffn = !fp8 && !invariant && any_swap && !any_normal && ffn_swap_supported(T, H, I) &&
+                       fused_ffn_enabled() && !(dbg && dbg->force_orient == 3);
+  if (use_ffn) {
+    GemmArgs a = g13;
+    a.chunks = at<int4>(ws, L.chunks_swap);
+    a.nchunks = hdr + kHdrChunksSwap;
+    a.mtiles = I / kTileM;
+    a.amax_cta = nullptr;
+    a.amax_n = 0;
+    a.flags = flags + 0 * kMaxSlots;
+    GemmArgs b = g2;
+    b.chunks = at<int4>(ws, L.chunks_swap);
+    b.nchunks = hdr + kHdrChunksSwap;
+    b.mtiles = H / kTileM;
+    b.flags = flags + 2 * kMaxSlots;
+    b.partials = at<float>(ws, L.partials2);
+    MOE_TRY(cuda_status(launch_ffn_swap(tw13s, txs, tw2s, tis, a, b, flags + kGemmLaunches * kMaxSlots, grid, st)));
+    record(dbg, 4, st);
+    record(dbg, 5, st);
+  } else {
+    if (any_swap) {
+      GemmArgs g = g13;
+      g.chunks = at<int4>(ws, L.chunks_swap);
+      g.nchunks = hdr + kHdrChunksSwap;
+      g.mtiles = I / kTileM;
+      g.amax_cta = amax_cta;
+      g.flags = flags + 0 * kMaxSlots;
+      requant_args(g, !any_normal);
+      MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW13, fp8, tw13s, txs, g, grid, st)));
+    }
+    if (any_normal) {
+      GemmArgs g = g13;
+      g.chunks = at<int4>(ws, L.chunks_pair);
+      g.nchunks = hdr + kHdrChunksPair;
+      g.mtiles = I / gemm_weight_box_rows(Orient::kNormal, Proj::kW13);
+      g.amax_cta = amax_cta + (any_swap ? grid : 0);
+      g.flags = flags + 1 * kMaxSlots;
+      requant_args(g, true);
+      MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
+    }
+    record(dbg, 4, st);   // (the FP8 requantisation ran at the end of the gate/up GEMM)
+    record(dbg, 5, st);
+    if (any_swap) {
+      GemmArgs g = g2;
+      g.chunks = at<int4>(ws, L.chunks_swap);
+      g.nchunks = hdr + kHdrChunksSwap;
+      g.mtiles = H / kTileM;
+      g.flags = flags + 2 * kMaxSlots;
+      MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, fp8, tw2s, tis, g, grid, st)));
+    }
+    if (any_normal) {
+      GemmArgs g = g2;
+      g.chunks = at<int4>(ws, L.chunks_normal);
+      g.nchunks = hdr + kHdrChunksNormal;
+      g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
+      g.flags = flags + 3 * kMaxSlots;
+      MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
+    }
   }
   record(dbg, 6, st);
   if (any_normal)
@@ -612,13 +645,12 @@ moe_status_t moe_align(const int32_t* topk_ids, int T, int E, int top_k, int32_t
     return MOE_ERR_UNSUPPORTED_SHAPE;
   if (!topk_ids || !counts || !offsets || !perm || !inv_perm || !workspace) return MOE_ERR_INVALID_ARG;
   const Layout L = make_layout(T, 128, E, 128, top_k, false);
-  if (workspace_bytes < L.gemm_flags + static_cast<size_t>(kGemmLaunches) * kMaxSlots * 4)
-    return MOE_ERR_WORKSPACE_TOO_SMALL;
+  if (workspace_bytes < L.gemm_flags + static_cast<size_t>(L.n_gemm_flags) * 4) return MOE_ERR_WORKSPACE_TOO_SMALL;
   AlignArgs aa{topk_ids, T, E, top_k, counts, offsets, perm, inv_perm,
                at<int4>(workspace, L.chunks_swap), at<int4>(workspace, L.chunks_normal),
                at<int4>(workspace, L.chunks_pair),
                swap_threshold(), gemm_swap_chunk(), nullptr, at<uint32_t>(workspace, L.header),
-               at<int>(workspace, L.gemm_flags), kGemmLaunches * kMaxSlots,
+               at<int>(workspace, L.gemm_flags), L.n_gemm_flags,
                at<int>(workspace, L.slice_hist)};
   return cuda_status(launch_align(aa, static_cast<cudaStream_t>(stream)));
 }

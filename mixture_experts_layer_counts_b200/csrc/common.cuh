@@ -22,6 +22,7 @@ enum WaitSite : uint32_t {
   kSiteDrainTma = 5,
   kSiteDrainMma = 6,
   kSiteGridBarrier = 7,
+  kSiteDependency = 8,     // fused FFN: a down-projection tile waited for its gate/up rows
 };
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
@@ -71,6 +72,8 @@ struct Layout {
   size_t header, topk_ids, topk_w, logits, xnorm, wnorm, amax_tok, amax_cta, cand, rsplit;
   size_t slice_hist;
   size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, chunks_pair, gemm_flags, partials;
+  size_t partials2;            // second set of partial tiles (the fused FFN's down GEMM)
+  int n_gemm_flags;            // split-tile flags of every GEMM launch + per-chunk counters
   size_t xperm, inter, h32, ysc, tickets, staging_in, staging_out, total;
   int max_chunks_swap, max_chunks_normal, max_chunks_pair;
 };
@@ -118,8 +121,12 @@ inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   L.chunks_normal = take(static_cast<size_t>(L.max_chunks_normal) * 16);
   L.max_chunks_pair = static_cast<int>(E + A / kPairTokens + 1);
   L.chunks_pair = take(static_cast<size_t>(L.max_chunks_pair) * 16);
-  L.gemm_flags = take(static_cast<size_t>(kGemmLaunches) * kMaxSlots * 4);
+  // flags of the GEMM launches, then one counter per swap-AB chunk (the fused
+  // FFN's gate/up -> down dependency); all zeroed by the align kernel
+  L.n_gemm_flags = kGemmLaunches * kMaxSlots + L.max_chunks_swap;
+  L.gemm_flags = take(static_cast<size_t>(L.n_gemm_flags) * 4);
   L.partials = take(static_cast<size_t>(kMaxSlots) * kPartialSlotFloats * 4);
+  L.partials2 = take(static_cast<size_t>(kMaxSlots) * kPartialSlotFloats * 4);
   const size_t eb = fp8 ? 1 : 2;
   L.xperm = take(A * H * eb);
   L.inter = take(A * I * eb);

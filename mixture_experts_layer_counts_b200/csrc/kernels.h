@@ -141,6 +141,14 @@ struct GemmArgs {
                                // element then sees the same operations whatever the batch
 };
 
+// Fused expert FFN of decode batches (ffn.cu): gate/up and down GEMMs, swap-AB,
+// bf16, one persistent launch; chunks of at most ffn_swap_chunk() tokens.
+bool ffn_swap_supported(int T, int H, int I);
+int ffn_swap_chunk();
+cudaError_t launch_ffn_swap(const CUtensorMap& tw13, const CUtensorMap& tx, const CUtensorMap& tw2,
+                            const CUtensorMap& th, const GemmArgs& g13, const GemmArgs& g2, int* dep, int grid,
+                            cudaStream_t st);
+
 enum class Orient { kSwap, kNormal };
 enum class Proj { kW13, kW2 };
 cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tm_w,

@@ -385,3 +385,20 @@ def cache_stats():
     v = (C.c_ulonglong * 4)()
     _lib.lib().moe_cache_stats(v)
     return dict(replays=v[0], captures=v[1], failures=v[2], direct=v[3])
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "decode-zipf"])
+def test_fused_ffn_matches_two_launch_path(cuda_ok, name):
+    # bf16 decode batches (T <= 32) run both GEMMs in one persistent launch;
+    # force_orient=3 runs the same swap-AB GEMMs as two launches.  Both meet
+    # the bound against the oracle and agree closely with each other (their
+    # split-K partial sums are grouped differently).
+    inp = make_inputs(WORKLOADS[name], "cuda")
+    fused, dbg_f = run(inp)
+    two, dbg_t = run(inp, force=3)
+    assert torch.equal(dbg_f["inter"].view(torch.int16), dbg_t["inter"].view(torch.int16))
+    ref = oracle_of(inp)
+    assert_output_close(fused, ref, fp8=False)
+    assert_output_close(two, ref, fp8=False)
+    d = (fused.float() - two.float()).abs().max().item()
+    assert d <= 2e-2 * max(ref["out"].std(), 1e-6), d
