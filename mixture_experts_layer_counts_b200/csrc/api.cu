@@ -164,6 +164,49 @@ void record(moe_debug_out_t* dbg, int i, cudaStream_t st) {
     cudaEventRecord(ev, st);
 }
 
+// Large batches: router logits on the tensor cores (the swap-AB kernel in its
+// dense router mode: expert rows in M, 64-token chunks of hidden in N, fp32
+// accumulation, whole units dealt round-robin), then the top-k kernel.  The
+// logits carry at most H * 2^-22 * ||x|| ||w|| of error: every MMA adds 16
+// exact bf16 products to the fp32 accumulator, and even an accumulation that
+// aligns them to the largest exponent and truncates loses at most 17 units in
+// the last place of the running magnitude per instruction (H / 16
+// instructions; a factor 2 of margin).  Tokens whose top-(k+1) gaps that
+// bound cannot separate are re-ranked in fp64, then exactly, as on every path.
+bool tc_router_eligible(int T, int H, int E, bool invariant) {
+  return !invariant && static_cast<double>(T) * E * H > static_cast<double>(1 << 28);
+}
+
+moe_status_t route_tc(const RouterArgs& ra, int grid, unsigned long long timeout_ns, cudaStream_t st) {
+  CUtensorMap tw, tx;
+  MOE_TRY(make_tmap(&tw, ra.router_w, false, ra.H, ra.E, gemm_weight_box_rows(Orient::kSwap, Proj::kW2)));
+  MOE_TRY(make_tmap(&tx, ra.hidden, false, ra.H, ra.T, gemm_token_box_rows(Orient::kSwap)));
+  GemmArgs g{};
+  g.dense_T = ra.T;
+  g.dense_chunk = gemm_swap_chunk();
+  g.n_cols = ra.E;
+  g.col_bias = ra.bias;
+  g.norm_x = ra.hidden;
+  g.norm_w = ra.router_w;
+  g.xnorm = ra.xnorm;
+  g.wnorm = ra.wnorm;
+  g.amax_tok = ra.amax_tok;
+  g.norm_H = ra.H;
+  g.mtiles = (ra.E + kTileM - 1) / kTileM;
+  g.katoms = ra.H * 2 / kAtomBytes;
+  g.w_rows_per_expert = 0;
+  g.out = ra.logits;
+  g.ld_out = ra.E;
+  g.num_assign = ra.T;
+  g.hdr = ra.hdr;
+  g.timeout_ns = timeout_ns;
+  g.whole_units = 1;
+  MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, false, tw, tx, g, grid, st)));
+  const float gamma = static_cast<float>(static_cast<double>(ra.H) * 2.384185791015625e-07);   // H * 2^-22
+  const float ulast = 5.9604644775390625e-08f;                                                 // the bias add
+  return cuda_status(launch_router_topk(ra, gamma, ulast, st));
+}
+
 moe_status_t forward_impl(const void* hidden, const void* router_w, const float* router_bias,
                           const void* w13, const void* w2, const float* w13_scale,
                           const float* w2_scale, int T, int H, int E, int I, int k, int dtype,
@@ -225,7 +268,14 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   // Decode-sized calls run logits, top-k and align in one launch (the
   // "router" stage then covers the align too and the "align" stage is empty).
   bool fused_route = false;
-  MOE_TRY(cuda_status(launch_router(ra, st, invariant ? nullptr : &aa, &fused_route)));
+  const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;
+  const unsigned long long timeout_ns = (dbg && dbg->wait_timeout_us > 0)
+                                            ? static_cast<unsigned long long>(dbg->wait_timeout_us) * 1000ull
+                                            : kWaitTimeoutNs;
+  if (tc_router_eligible(T, H, E, invariant))
+    MOE_TRY(route_tc(ra, grid, timeout_ns, st));
+  else
+    MOE_TRY(cuda_status(launch_router(ra, st, invariant ? nullptr : &aa, &fused_route)));
   record(dbg, 1, st);
   if (!fused_route) MOE_TRY(cuda_status(launch_align(aa, st)));
   record(dbg, 2, st);
@@ -234,7 +284,6 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                                     A, k, H, fp8, hdr, xperm, st)));
   record(dbg, 3, st);
 
-  const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;
   int* flags = at<int>(ws, L.gemm_flags);   // one kMaxSlots array per GEMM launch
   GemmArgs g13{};
   g13.katoms = H * (fp8 ? 1 : 2) / kAtomBytes;
@@ -250,9 +299,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g13.act_scale = hdr + kHdrScaleS1;
   g13.hdr = hdr;
   g13.partials = at<float>(ws, L.partials);
-  g13.timeout_ns = (dbg && dbg->wait_timeout_us > 0)
-                       ? static_cast<unsigned long long>(dbg->wait_timeout_us) * 1000ull
-                       : kWaitTimeoutNs;
+  g13.timeout_ns = timeout_ns;
   g13.inject_stall = dbg ? dbg->inject_stall : 0;
   g13.whole_units = invariant ? 1 : 0;
   float* amax_cta = at<float>(ws, L.amax_cta);
@@ -634,6 +681,10 @@ moe_status_t moe_route(const void* hidden, const void* router_w, const float* ro
                 at<float>(workspace, L.wnorm), at<float>(workspace, L.amax_tok), topk_ids, topk_w,
                 at<unsigned char>(workspace, L.cand), at<uint32_t>(workspace, L.header),
                 at<float>(workspace, L.rsplit)};
+  if (tc_router_eligible(T, H, E, false)) {
+    const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;
+    return route_tc(ra, grid, kWaitTimeoutNs, static_cast<cudaStream_t>(stream));
+  }
   return cuda_status(launch_router(ra, static_cast<cudaStream_t>(stream)));
 }
 

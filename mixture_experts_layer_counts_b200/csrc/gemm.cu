@@ -182,8 +182,10 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
   // wait for its predecessors.  So the schedule may be read, and the weight
   // tiles (inputs of the call, written by no kernel) fetched, before the wait
   // for the previous kernel's activations.
-  const long long nunits =
-      static_cast<long long>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks)) * a.mtiles;
+  const long long nchunks =
+      a.dense_T > 0 ? (a.dense_T + a.dense_chunk - 1) / a.dense_chunk
+                    : static_cast<long long>(*reinterpret_cast<const volatile uint32_t*>(a.nchunks));
+  const long long nunits = nchunks * a.mtiles;
   const int ksteps = a.katoms / KA;   // pipeline stages per unit
   const long long W = nunits * ksteps;
   // Swap-AB: contiguous balanced atom ranges (units may be split across CTAs).
@@ -404,6 +406,42 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     const int row = q * 32 + lane;        // accumulator row held by this thread
     float amax = 0.f;
     int it = 0;
+    if (a.dense_T > 0 && a.xnorm != nullptr) {
+      // router logits: while the first tiles stream in, these warps write the
+      // norms and amax of a grid-strided share of the token and router rows
+      const int vpr = a.norm_H / 8;
+      const long long rows = static_cast<long long>(a.dense_T) + a.n_cols;
+      for (long long r = static_cast<long long>(blockIdx.x) * C::kEpiWarps + (warp - 2); r < rows;
+           r += static_cast<long long>(gridDim.x) * C::kEpiWarps) {
+        const bool tok = r < a.dense_T;
+        const uint4* src = static_cast<const uint4*>(tok ? a.norm_x : a.norm_w) +
+                           static_cast<size_t>(tok ? r : r - a.dense_T) * vpr;
+        float ss = 0.f, am = 0.f;
+        for (int c = lane; c < vpr; c += 32) {
+          const uint4 v4 = src[c];
+          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f2 = __bfloat1622float2(b2[i]);
+            ss = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, ss));
+            am = fmaxf(am, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+          }
+        }
+#pragma unroll
+        for (int m = 16; m > 0; m >>= 1) {
+          ss += __shfl_xor_sync(0xffffffffu, ss, m);
+          am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, m));
+        }
+        if (lane == 0) {
+          if (tok) {
+            a.xnorm[r] = sqrtf(ss);
+            a.amax_tok[r] = am;
+          } else {
+            a.wnorm[r - a.dense_T] = sqrtf(ss);
+          }
+        }
+      }
+    }
     Segments seg = seg0;
     int u, kb0, kb1;
     while (seg.next(u, kb0, kb1)) {
@@ -498,17 +536,34 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
         }
       } else if constexpr (C::kSwap) {
         const int hrow = mt * kTileM + row;
-        for (int c0 = 0; c0 < ncols; c0 += 16) {
-          float v[1][16];
-          tmem_ld16_wait(tbase + c0, v[0]);
-          add_partials(v, c0);
+        if (a.dense_T > 0) {
+          // router logits: row = expert, column n = token p0 + n
+          const bool live = hrow < a.n_cols;
+          const float b = (live && a.col_bias != nullptr) ? a.col_bias[hrow] : 0.f;
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float v[1][16];
+            tmem_ld16_wait(tbase + c0, v[0]);
+            add_partials(v, c0);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            const int f = n < nv ? a.perm[p0 + n] : -1;
-            if (f >= 0 && f < a.num_assign) {
-              const float wt = a.topk_w[f];
-              static_cast<float*>(a.out)[static_cast<size_t>(f) * a.ld_out + hrow] = v[0][j] * scale * wt;
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              if (live && n < nv)
+                static_cast<float*>(a.out)[static_cast<size_t>(p0 + n) * a.ld_out + hrow] = v[0][j] + b;
+            }
+          }
+        } else {
+          for (int c0 = 0; c0 < ncols; c0 += 16) {
+            float v[1][16];
+            tmem_ld16_wait(tbase + c0, v[0]);
+            add_partials(v, c0);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int n = c0 + j;
+              const int f = n < nv ? a.perm[p0 + n] : -1;
+              if (f >= 0 && f < a.num_assign) {
+                const float wt = a.topk_w[f];
+                static_cast<float*>(a.out)[static_cast<size_t>(f) * a.ld_out + hrow] = v[0][j] * scale * wt;
+              }
             }
           }
         }

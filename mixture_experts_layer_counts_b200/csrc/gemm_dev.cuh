@@ -61,6 +61,12 @@ template <bool kGrouped, int kChunkTokens>
 __device__ __forceinline__ void unit_coords(const GemmArgs& a, int u, int4& ch, int& mt) {
   const int cs = u / a.mtiles;   // a chunk of the unit's expert
   if constexpr (!kGrouped) {
+    if (a.dense_T > 0) {   // router logits: dense chunks of dense_chunk hidden rows
+      mt = u - cs * a.mtiles;
+      const int n0 = cs * a.dense_chunk;
+      ch = make_int4(0, n0, min(a.dense_chunk, a.dense_T - n0), cs);
+      return;
+    }
     ch = a.chunks[cs];
     mt = u - cs * a.mtiles;
   } else {

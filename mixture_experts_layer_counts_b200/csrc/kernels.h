@@ -66,6 +66,10 @@ struct AlignArgs;
 // one launch (then *fused is set and the align must not be launched again).
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align = nullptr,
                           bool* fused = nullptr);
+// The router's top-k kernel alone (logits, norms and amax already written),
+// with the relative error bound `gamma` of the logits (times ||x|| ||w||) and
+// `ulast` of their last roundings.
+cudaError_t launch_router_topk(const RouterArgs& a, float gamma, float ulast, cudaStream_t st);
 
 struct AlignArgs {
   const int32_t* topk_ids;
@@ -136,6 +140,21 @@ struct GemmArgs {
   void* y_out;                 // w2: out [T, H], written by the combine in the epilogue:
   int y_fp32;                  //   bf16 (0), or the unrounded fp32 sum (1, tensor-parallel partials)
   int top_k;
+  // Router logits mode of the swap-AB down-projection kernel (dense_T > 0):
+  // weight rows = router rows (n_cols experts), token chunks = dense tiles of
+  // the hidden rows (no schedule, no perm), out = logits [dense_T, n_cols] fp32
+  // with col_bias added; the epilogue warps first write the norms the
+  // router's certification needs (||x_t||, amax|x_t|, ||w_e||).
+  int dense_T;
+  int dense_chunk;             // tokens per dense chunk (the swap-AB kernel's largest N)
+  int n_cols;
+  const float* col_bias;
+  const void* norm_x;          // hidden [dense_T, norm_H] bf16
+  const void* norm_w;          // router_w [n_cols, norm_H] bf16
+  float* xnorm;
+  float* wnorm;
+  float* amax_tok;
+  int norm_H;
   int whole_units;             // 1: whole units dealt round-robin (no K splits) and, for
                                // swap-AB, MMA N fixed at the largest chunk: every output
                                // element then sees the same operations whatever the batch

@@ -923,6 +923,13 @@ static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStre
                     a.logits, a.xnorm, a.wnorm, a.amax_tok, a.rsplit);
 }
 
+cudaError_t launch_router_topk(const RouterArgs& a, float gamma, float ulast, cudaStream_t st) {
+  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, 1, st);
+  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, 1, st);
+  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, 1, st);
+  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, 1, st);
+}
+
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align, bool* fused) {
   if (fused) *fused = false;
   // fp64 accumulation while the logit work is small (decode batches); fp32
