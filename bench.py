@@ -295,18 +295,20 @@ SWAP_MAX_TOKENS = 64   # the library's default swap-AB / normal threshold (token
 
 
 def launches_per_step(wl, T):
-    """Kernels one layer call launches: router (logits, top-k), align (two
-    slice grids from T*k = 8192 on), gather, w13 and w2 GEMMs (one per
-    orientation in use; the FP8 requantisation closes the last w13 launch),
-    and the combine pass when normal-orientation experts are present (else
-    the w2 epilogue combines)."""
+    """Kernels one layer call launches: router (logits, top-k, align: one
+    launch at decode sizes, else two plus one or two align grids), gather,
+    w13 and w2 GEMMs (one per orientation in use, or one fused launch for
+    bf16 decode batches; the FP8 requantisation closes the last w13 launch),
+    and the combine pass."""
     any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
     A = T * wl["top_k"]
     # decode-sized calls: logits, top-k and align in one launch
     fused_router = A < 8192 and wl["E"] <= 256
     n_route = 1 if fused_router else 2 + (2 if A >= 8192 else 1)
-    # with normal-orientation experts the combine is a separate pass
-    return n_route + 1 + 2 * (2 if any_normal else 1) + (1 if any_normal else 0)
+    # bf16 decode batches (T <= 32): both GEMMs in one launch; then the combine pass
+    fused_ffn = wl["dtype"] == "bf16" and T <= 32 and os.environ.get("MOE_FUSED_FFN", "1") != "0"
+    n_gemm = 1 if fused_ffn else 2 * (2 if any_normal else 1)
+    return n_route + 1 + n_gemm + 1
 
 
 def new_events(n, stream):

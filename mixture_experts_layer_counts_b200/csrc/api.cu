@@ -257,8 +257,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 router_bias, T, H, E, k,
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
-                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0,
-                at<int>(ws, L.tickets)};
+                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0};
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
@@ -323,14 +322,6 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   g2.amax_cta = nullptr;
   g2.amax_n = 0;
   g2.inject_stall = 0;
-  // Combine: when every expert runs swap-AB (decode batches) the down GEMM's
-  // epilogue combines (tickets); with normal-orientation experts the slot rows
-  // are summed by a separate pass (the epilogue's combine reads would then
-  // compete with the tensor-bound mainloop; measured slower)
-  g2.tickets = any_normal ? nullptr : at<int>(ws, L.tickets);   // zeroed by the router's top-k kernel
-  g2.y_out = out;
-  g2.y_fp32 = out_fp32 ? 1 : 0;
-  g2.top_k = k;
   // Decode batches in bf16 (T <= 32, every expert swap-AB): both GEMMs in one
   // persistent launch (ffn.cu); otherwise one launch per GEMM and orientation.
   const bool use_ffn = !fp8 && !invariant && any_swap && !any_normal && ffn_swap_supported(T, H, I) &&
@@ -393,8 +384,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     }
   }
   record(dbg, 6, st);
-  if (any_normal)
-    MOE_TRY(cuda_status(launch_combine(at<float>(ws, L.ysc), T, k, H, out, out_fp32, st)));
+  // combine: out[t] = sum_j ysc[t*k + j] in slot order (fp32), one rounding
+  MOE_TRY(cuda_status(launch_combine(at<float>(ws, L.ysc), T, k, H, out, out_fp32, st)));
   record(dbg, 7, st);
 
   if (dbg) {

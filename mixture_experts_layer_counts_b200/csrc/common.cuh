@@ -35,7 +35,6 @@ constexpr int kTokenBox = 16;          // rows per TMA box of the token operand 
 constexpr int kNormalTokens = 128;     // token rows per tile in normal orientation (M)
 constexpr int kPairTokens = 256;       // gate/up GEMM, normal orientation: two M tiles per weight tile
 constexpr int kMaxTopK = 32;
-constexpr int kTicketCols = 128;        // output columns per combine ticket (one per token and tile)
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxGrid = 1024;          // persistent grids never exceed this
 constexpr int kMaxSlots = 160;          // GEMM CTAs per launch (>= the SM count of a B200)
@@ -74,7 +73,7 @@ struct Layout {
   size_t counts, offsets, perm, inv_perm, chunks_swap, chunks_normal, chunks_pair, gemm_flags, partials;
   size_t partials2;            // second set of partial tiles (the fused FFN's down GEMM)
   int n_gemm_flags;            // split-tile flags of every GEMM launch + per-chunk counters
-  size_t xperm, inter, h32, ysc, tickets, staging_in, staging_out, total;
+  size_t xperm, inter, h32, ysc, staging_in, staging_out, total;
   int max_chunks_swap, max_chunks_normal, max_chunks_pair;
 };
 
@@ -132,7 +131,6 @@ inline Layout make_layout(int T, int H, int E, int I, int k, bool fp8) {
   L.inter = take(A * I * eb);
   L.h32 = fp8 ? take(A * I * 4) : off;
   L.ysc = take(A * H * 4);
-  L.tickets = take(static_cast<size_t>(T) * (H / kTicketCols) * 4);
   L.staging_in = take(static_cast<size_t>(T) * H * 2);
   L.staging_out = take(static_cast<size_t>(T) * H * 2);
   L.total = off;

@@ -1,6 +1,6 @@
 // Fused expert FFN of decode batches: the gate/up GEMM (SiLU * up epilogue)
-// and the down GEMM (router-weighted slot rows and the in-epilogue combine)
-// in one persistent launch, swap-AB orientation, bf16.
+// and the down GEMM (router-weighted slot rows) in one persistent launch,
+// swap-AB orientation, bf16.
 //
 // Why.  At decode every active expert's weights are streamed once and the
 // layer is bound by HBM; between two launches the first GEMM's tail (CTAs
@@ -49,14 +49,12 @@ constexpr int kFfnBN = 32;                                   // largest token ch
 constexpr int kFfnATile = kTileM * kAtomBytes;               // 128 weight rows x 128 B
 constexpr int kFfnBTile = kFfnBN * kAtomBytes;               // 32 token rows x 128 B
 constexpr int kFfnStage = 2 * (kFfnATile + kFfnBTile);       // 40 KB
-constexpr int kFfnCombList = 64;
-constexpr int kFfnCombBytes = 2 * (kFfnCombList + 4) * 4;
-constexpr int kFfnStages = (232448 - 1280 - kFfnCombBytes) / kFfnStage;
+constexpr int kFfnStages = (232448 - 1280) / kFfnStage;
 constexpr int kFfnThreads = 192;
 constexpr int kFfnEpiWarps = 4;
 constexpr int kFfnAccCols = 2 * kFfnBN;                      // per TMEM buffer: gate + up
 constexpr int kFfnTmemCols = 2 * kFfnAccCols;                // two buffers
-constexpr int kFfnSmem = kFfnStages * kFfnStage + 1024 + 256 + kFfnCombBytes;
+constexpr int kFfnSmem = kFfnStages * kFfnStage + 1024 + 256;
 static_assert(kFfnStages >= 4, "pipeline depth");
 static_assert(kFfnSmem <= 232448, "shared memory");
 
@@ -123,7 +121,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
   uint64_t* drain = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* comb = reinterpret_cast<int*>(tiles + kFfnStages * kFfnStage + 256);
 
   const GemmArgs& a1 = f.g13;
   const GemmArgs& a2 = f.g2;
@@ -371,7 +368,7 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
     constexpr int kEpiThreads = 32 * kFfnEpiWarps;
     const int q = warp & 3;
     const int row = q * 32 + lane;
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - 64;   // 0 .. kEpiThreads - 1
     int it = 0;
     bool ok = true;
     for (int ph = 0; ph < 2 && ok; ++ph) {
@@ -490,24 +487,6 @@ __global__ void __launch_bounds__(kFfnThreads, 1)
           // precedes the barrier; one release increment of the chunk's count
           epilogue_bar<kEpiThreads>();
           if (et == 0) red_release_add(f.dep + cs, 1);
-        } else if (a.tickets != nullptr) {
-          // combine: the CTA that writes a token's last slot of this tile sums it
-          int* list = comb + (it & 1) * (kFfnCombList + 4);
-          int* nlist = list + kFfnCombList;
-          if (et == 0) *nlist = 0;
-          epilogue_bar<kEpiThreads>();
-          if (et < nv) {
-            const int fl = a.perm[p0 + et];
-            if (fl >= 0 && fl < a.num_assign) {
-              const int t = fl / a.top_k;
-              const int ntile = a.ld_out / kTicketCols;
-              if (atom_add_acq_rel(a.tickets + static_cast<size_t>(t) * ntile + mt, 1) == a.top_k - 1)
-                list[atomicAdd(nlist, 1)] = t * 64 + mt;
-            }
-          }
-          epilogue_bar<kEpiThreads>();
-          const int nl = *nlist;
-          for (int i = warp - 2; i < nl; i += kFfnEpiWarps) combine_tile(a, list[i] >> 6, list[i] & 63, lane);
         }
       }
     }

@@ -25,13 +25,8 @@
 //          grid barrier and the per-tensor E4M3 requantisation of h
 //          (requant_tail), so no separate pass is launched.
 //   kW2  : one accumulator; the epilogue multiplies by the router weight
-//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot).  When
-//          every expert of the call runs swap-AB (decode batches), it then
-//          takes an integer ticket per (token, 128-column tile); the CTA that
-//          writes a token's last slot of a tile sums the k slot rows in slot
-//          order and writes the output (combine_tile), so the combine runs
-//          inside this kernel; otherwise a separate pass sums the slot rows in
-//          the same order.  Deterministic, no floating-point atomics.
+//          w[t, j] and writes the fp32 row to ysc[t*k + j] (its slot), which
+//          the combine pass sums in slot order: deterministic, no atomics.
 //
 // Work split.  A "unit" is one output tile (token chunk x weight-row tile)
 // and needs `katoms` K atoms.
@@ -105,18 +100,14 @@ struct Cfg {
   static constexpr int kEpiCols = 16;
   static constexpr int kEpiLd = 20;
   static constexpr int kEpiBytes = kSwap ? 0 : kEpiWarps * 32 * kEpiLd * 4;
-  // w2: two lists (units alternate) of the (token, tile) pairs whose combine
-  // this CTA completes, at most 2 * kTileM per unit, plus their lengths
-  static constexpr int kCombList = 2 * kTileM;
-  static constexpr int kCombBytes = kDual ? 0 : 2 * (kCombList + 4) * 4;
-  static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes - kCombBytes) / kStageBytes;
+  static constexpr int kStagesFit = (232448 - 1280 - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kNumAcc = kDual ? 2 : 1;
   static constexpr int kAccCols = kNumAcc * kBN * (kPair ? 2 : 1);   // per TMEM buffer
   static constexpr int kAccBufs = kPair ? 1 : 2;               // pair: 512 columns, one buffer
   static constexpr int kTmemCols = kAccBufs * kAccCols;        // 128, 256 or 512
   static constexpr int kSmemBytes =
-      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes + kCombBytes;
+      kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/ + kEpiBytes;
   static constexpr int kAtomElems = FP8 ? 128 : 64;
   static constexpr int kSlotFloats = kNumAcc * kTileM * kBN;   // one CTA's partial tile
   static_assert(kTmemCols >= 32 && kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0,
@@ -146,7 +137,6 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* red = reinterpret_cast<float*>(tmem_slot + 2);   // per epilogue warp amax (<= 8)
   float* epi = reinterpret_cast<float*>(smem + C::kStages * C::kStageBytes + 256);
-  int* comb = reinterpret_cast<int*>(smem + C::kStages * C::kStageBytes + 256 + C::kEpiBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -670,48 +660,6 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
-
-      if constexpr (!C::kDual) {
-        // ---- combine: a token's output tile is summed by the CTA that
-        // writes the last of its k slot pieces.  After a barrier of the
-        // epilogue warps (every slot row of the unit stored), one thread per
-        // (token, tile) of the unit takes a ticket with release/acquire
-        // semantics; the thread that draws k - 1 lists the pair, and the
-        // epilogue warps sum the listed pairs, reading through L2.  Integer
-        // tickets only; the sums run in slot order, so the result does not
-        // depend on which CTA finishes last.
-        if (a.tickets != nullptr) {
-          constexpr int kEpiThreads = 32 * C::kEpiWarps;
-          const int et = threadIdx.x - 64;          // 0 .. kEpiThreads - 1
-          int* list = comb + (it & 1) * (C::kCombList + 4);
-          int* nlist = list + C::kCombList;
-          if (et == 0) *nlist = 0;
-          // every epilogue thread's slot-row stores precede the barrier; the
-          // ticket's release (acq_rel at GPU scope) publishes them with it
-          epilogue_bar<kEpiThreads>();
-          // swap-AB: one tile (the unit's 128 H rows), tokens n < nv;
-          // normal: two tiles (256 H columns), tokens r < nv
-          const int r = C::kSwap ? et : (et & (kTileM - 1));
-          const int tile = C::kSwap ? mt : 2 * mt + (et >> 7);
-          if (r < nv && (C::kSwap ? et < kTileM : true)) {
-            const int f = a.perm[p0 + r];
-            if (f >= 0 && f < a.num_assign) {
-              const int t = f / a.top_k;
-              const int ntile = a.ld_out / kTicketCols;
-              if (atom_add_acq_rel(a.tickets + static_cast<size_t>(t) * ntile + tile, 1) == a.top_k - 1)
-                list[atomicAdd(nlist, 1)] = t * 64 + tile;
-            }
-          }
-          epilogue_bar<kEpiThreads>();
-          const int n = *nlist;
-          if (n > 0) {
-            for (int i = (warp - 2); i < n; i += C::kEpiWarps) {
-              const int v = list[i];
-              combine_tile(a, v >> 6, v & 63, lane);
-            }
-          }
-        }
-      }
     }
     if constexpr (FP8 && C::kDual) {
 #pragma unroll

@@ -1,7 +1,6 @@
 // Device helpers shared by the grouped GEMM kernels (gemm.cu) and the fused
 // swap-AB expert FFN kernel (ffn.cu): the stream-K work split, the unit ->
-// tile mapping, bounded flag waits, the in-epilogue combine and the FP8
-// requantisation tail.
+// tile mapping, bounded flag waits and the FP8 requantisation tail.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -114,52 +113,6 @@ __device__ __forceinline__ bool wait_flag(const int* flag, volatile int* abort, 
       }
     }
   }
-}
-
-__device__ __forceinline__ int atom_add_acq_rel(int* p, int v) {
-  int old;
-  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
-// Combine of one (token t, ticket tile) pair by one warp: out[t, tile cols] =
-// bf16( sum_{j < k} ysc[t*k + j, tile cols] ), the fp32 sum in slot order
-// j = 0, 1, ... (the definition's order), 4 columns per lane.  The slot rows
-// were written by other CTAs: read through L2.
-__device__ __forceinline__ void combine_tile(const GemmArgs& a, int t, int tile, int lane) {
-  const int H = a.ld_out;
-  const int col = tile * kTicketCols + lane * 4;
-  const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.out) +
-                                                      static_cast<size_t>(t) * a.top_k * H + col);
-  const size_t stride = static_cast<size_t>(H) / 4;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j0 = 0; j0 < a.top_k; j0 += 8) {
-    float4 y[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u)
-      if (j0 + u < a.top_k) y[u] = __ldcg(src + static_cast<size_t>(j0 + u) * stride);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (j0 + u < a.top_k) {
-        if (j0 + u == 0) {
-          acc = y[u];
-        } else {
-          acc.x += y[u].x;
-          acc.y += y[u].y;
-          acc.z += y[u].z;
-          acc.w += y[u].w;
-        }
-      }
-    }
-  }
-  if (a.y_fp32) {   // tensor-parallel partial: the unrounded sum
-    *reinterpret_cast<float4*>(static_cast<float*>(a.y_out) + static_cast<size_t>(t) * H + col) = acc;
-    return;
-  }
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.y_out) + static_cast<size_t>(t) * H + col) =
-      make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
 }
 
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {

@@ -59,7 +59,6 @@ struct RouterArgs {
   uint32_t* hdr;
   float* rsplit;          // router_split_floats(T, E) floats, or NULL (no split-K)
   int invariant;          // 1: one logits kernel and summation order for every T (no split-K)
-  int* tickets;           // [T, H / kTicketCols] combine tickets, zeroed by the top-k kernel (may be NULL)
 };
 struct AlignArgs;
 // fuse_align non-NULL: a decode-sized call may run logits, top-k and align in
@@ -136,10 +135,6 @@ struct GemmArgs {
   int* flags;                  // kMaxSlots flags, zero at launch
   unsigned long long timeout_ns;   // limit of every bounded wait in the kernel
   int inject_stall;            // failure-path test: CTA 0 leaves one stage unfilled
-  int* tickets;                // w2: [T, H / kTicketCols] combine tickets (zero at launch)
-  void* y_out;                 // w2: out [T, H], written by the combine in the epilogue:
-  int y_fp32;                  //   bf16 (0), or the unrounded fp32 sum (1, tensor-parallel partials)
-  int top_k;
   // Router logits mode of the swap-AB down-projection kernel (dense_T > 0):
   // weight rows = router rows (n_cols experts), token chunks = dense tiles of
   // the hidden rows (no schedule, no perm), out = logits [dense_T, n_cols] fp32

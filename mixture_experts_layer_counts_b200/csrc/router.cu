@@ -736,13 +736,11 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
-    uint32_t* __restrict__ hdr, int* __restrict__ tickets) {
+    uint32_t* __restrict__ hdr) {
   pdl_wait();
   pdl_launch_next();
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t >= T) return;
-  if (tickets != nullptr)   // this token's combine tickets start the call at zero
-    for (int i = threadIdx.x & 31; i < H / kTicketCols; i += 32) tickets[static_cast<size_t>(t) * (H / kTicketCols) + i] = 0;
   topk_token<kPer>(t, logits, xnorm, wnorm, amax_tok, rsplit, nsplit, bias, hidden, router_w, T, H,
                    E, k, gamma, ulast, topk_ids, topk_w, cand, hdr);
 }
@@ -789,9 +787,6 @@ __global__ void __launch_bounds__(256) router_fused_kernel(RouterArgs ra, AlignA
   const int nt = min(TT, ra.T - t0);
   for (int tt = threadIdx.x >> 5; tt < nt; tt += blockDim.x >> 5) {
     const int t = t0 + tt;
-    if (ra.tickets != nullptr)
-      for (int i = threadIdx.x & 31; i < ra.H / kTicketCols; i += 32)
-        ra.tickets[static_cast<size_t>(t) * (ra.H / kTicketCols) + i] = 0;
     topk_token<kPer>(t, ra.logits, ra.xnorm, ra.wnorm, ra.amax_tok, ra.rsplit, 1, ra.bias, ra.hidden,
                      ra.router_w, ra.T, ra.H, ra.E, ra.k, gamma, ulast, ra.topk_ids, ra.topk_w, ra.cand, ra.hdr);
   }
@@ -838,7 +833,7 @@ static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, in
                                cudaStream_t st) {
   return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
                     a.xnorm, a.wnorm, a.amax_tok, a.rsplit, nsplit, a.bias, a.hidden, a.router_w,
-                    a.T, a.H, a.E, a.k, gamma, ulast, a.topk_ids, a.topk_w, a.cand, a.hdr, a.tickets);
+                    a.T, a.H, a.E, a.k, gamma, ulast, a.topk_ids, a.topk_w, a.cand, a.hdr);
 }
 
 // ---------------------------------------------------------------------------

@@ -44,7 +44,9 @@ def test_inv_rope_fp8_bit_exact(cuda_ok, T, nH, D):
     codes, scales, pos = run_case(T, nH, D, 4096, seed=T + nH + D)
     if T > 4:
         assert not codes[1].any() and not codes[2].any() and not scales[1].any() and not scales[2].any()
-        assert scales[4, 0] == 1.0 and not codes[4, 0].any()
+        # an all-zero head: scale 1 and codes of +0 or -0 (a zero rotated by a
+        # negative sine is -0, code 0x80)
+        assert scales[4, 0] == 1.0 and not (codes[4, 0] & 0x7F).any()
 
 
 def test_inv_rope_fp8_large_call_sampled(cuda_ok):
