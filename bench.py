@@ -295,16 +295,15 @@ SWAP_MAX_TOKENS = 64   # the library's default swap-AB / normal threshold (token
 
 
 def launches_per_step(wl, T):
-    """Kernels one layer call launches: router (logits, top-k, align: one
-    launch at decode sizes, else two plus one or two align grids), gather,
+    """Kernels one layer call launches: router (logits and top-k; at decode
+    sizes the top-k's last CTA aligns, else one or two align grids), gather,
     w13 and w2 GEMMs (one per orientation in use, or one fused launch for
     bf16 decode batches; the FP8 requantisation closes the last w13 launch),
     and the combine pass."""
     any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
     A = T * wl["top_k"]
-    # decode-sized calls: logits, top-k and align in one launch
-    fused_router = A < 8192 and wl["E"] <= 256
-    n_route = 1 if fused_router else 2 + (2 if A >= 8192 else 1)
+    # logits, top-k (decode-sized calls: its last CTA aligns), else align (one or two grids)
+    n_route = 2 + (0 if (A < 8192 and wl["E"] <= 256) else (2 if A >= 8192 else 1))
     # bf16 decode batches (T <= 32): both GEMMs in one launch; then the combine pass
     fused_ffn = wl["dtype"] == "bf16" and T <= 32 and os.environ.get("MOE_FUSED_FFN", "1") != "0"
     n_gemm = 1 if fused_ffn else 2 * (2 if any_normal else 1)
@@ -598,6 +597,53 @@ def measure_inv_rope(local, steps=200):
             "tokens_per_s": T / (ms * 1e-3), "steps": steps}
 
 
+def sweep_orientation(local, counts=(8, 16, 24, 32, 48, 64, 80, 96, 128, 160, 192, 256), reps=20):
+    """Gate/up and down GEMM time under forced swap-AB and forced normal
+    orientation, for E = 16 experts holding exactly c tokens each (a one-hot
+    router sends token t to expert t mod 16, top_k = 1), H = 4096, I = 1536,
+    bf16.  Each GEMM timed by the library's stage events, L2 flushed before
+    every call; median of `reps` calls.  One JSON line per c."""
+    from mixture_experts_layer_counts_b200 import layer
+
+    H, I, E, k = 4096, 1536, 16, 1
+    dev = torch.device("cuda", local)
+    g = torch.Generator(device=dev).manual_seed(0)
+    w13 = (torch.randn(E, 2 * I, H, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    w2 = (torch.randn(E, H, I, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    router_w = torch.zeros(E, H, device=dev)
+    router_w[torch.arange(E), torch.arange(E)] = 1.0
+    router_w = router_w.to(torch.bfloat16)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for c in counts:
+        T = E * c
+        hidden = torch.randn(T, H, generator=g, device=dev) * 0.1
+        hidden[:, :E] = 0.0
+        idx = torch.arange(T, device=dev)
+        hidden[idx, idx % E] = 8.0
+        hidden = hidden.to(torch.bfloat16)
+        ws = layer.make_workspace(T, H, E, I, k, 0, dev)
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+        row = {"tokens_per_expert": c}
+        for force, name in ((1, "swap"), (2, "normal")):
+            evs = new_events(8, torch.cuda.current_stream(dev))
+            t13, t2 = [], []
+            for it in range(reps + 3):
+                flush.zero_()
+                layer.moe_forward(hidden, router_w, None, w13, w2, k, out=out, workspace=ws, force_orient=force,
+                                  stage_events=evs)
+                torch.cuda.synchronize()
+                if it >= 3:
+                    t13.append(evs[3].elapsed_time(evs[4]) * 1e3)
+                    t2.append(evs[5].elapsed_time(evs[6]) * 1e3)
+            dbg = {}
+            layer.moe_forward(hidden, router_w, None, w13, w2, k, debug=dbg)
+            cnt = dbg["counts"].cpu()
+            assert int(cnt.min()) == c and int(cnt.max()) == c, "routing did not give c tokens per expert"
+            row[name + "_w13_us"] = statistics.median(t13)
+            row[name + "_w2_us"] = statistics.median(t2)
+        print(json.dumps(row), flush=True)
+
+
 def run_ours(args, wl, rank, world, local):
     pk = peaks()
     head, cpu = measure_workload(args.workload, wl, args, rank, world, local, steps_exact=args.steps)
@@ -645,6 +691,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only-headline", action="store_true", help="skip the other workloads")
+    ap.add_argument("--sweep-orientation", action="store_true",
+                    help="time both GEMMs under forced swap-AB / normal orientation over tokens per expert")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch-invariant", action="store_true",
                     help="time moe_forward_batch_invariant (bf16 workloads)")
@@ -671,6 +719,9 @@ def main():
     args.steps = 200 if args.steps is None else args.steps
     args.warmup = 10 if args.warmup is None else args.warmup
     rank, world, local = dist_setup(args.gpus)
+    if args.sweep_orientation:
+        sweep_orientation(local)
+        return
     try:
         run_ours(args, wl, rank, world, local)
     finally:

@@ -264,7 +264,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                at<int4>(ws, L.chunks_pair),
                tau, gemm_swap_chunk(), fp8 ? at<float>(ws, L.amax_tok) : nullptr, hdr,
                at<int>(ws, L.gemm_flags), L.n_gemm_flags, at<int>(ws, L.slice_hist)};
-  // Decode-sized calls run logits, top-k and align in one launch (the
+  // Decode-sized calls: the top-k kernel's last CTA runs the align (the
   // "router" stage then covers the align too and the "align" stage is empty).
   bool fused_route = false;
   const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;

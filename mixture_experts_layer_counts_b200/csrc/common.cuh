@@ -51,14 +51,10 @@ constexpr int kHdrChunksPair = 7;      // number of normal-orientation 256-token
 constexpr int kHdrScaleS1 = 8;         // fp32 bits: activation scale (FP8)
 constexpr int kHdrScaleS2 = 9;         // fp32 bits: intermediate scale (FP8)
 constexpr int kHdrBarrier = 12;        // grid barrier counter
-constexpr int kStatusBytes = 256;      // the words above
-// Ticket counters of the fused decode router (self-resetting, zeroed once by
-// moe_workspace_init): word kHdrRouterAll counts finished token tiles, words
-// kHdrRouterTiles + i count the finished expert groups of token tile i.
-constexpr int kHdrRouterAll = 64;
-constexpr int kHdrRouterTiles = 128;
-constexpr int kRouterFusedMaxTiles = 8192;
-constexpr int kHeaderBytes = 65536;    // status words + router counters
+constexpr int kHdrRouterAll = 13;      // top-k CTAs finished (decode calls: the last one aligns;
+                                       // reset by that CTA, so every call starts at 0)
+constexpr int kHeaderBytes = 256;
+constexpr int kStatusBytes = kHeaderBytes;
 
 __device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, uint32_t where) {
   if (atomicCAS(status + kHdrStatus, 0u, code) == 0u) {

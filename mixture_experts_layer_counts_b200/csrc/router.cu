@@ -141,35 +141,44 @@ __device__ __forceinline__ int exact_cmp(const long long (&a)[kLimbs], const lon
   return 0;
 }
 
-// fp64 logit (tier 2): exact products, four fp64 partial sums per lane (four
-// loads in flight), then the butterfly.  Every term passes through at most
-// H/32 + 8 roundings, inside the H/32 + 16 the bound assumes.
-__device__ double fp64_logit(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* __restrict__ w,
-                             int H) {
+// Up to four fp64 logits of one token row at once (tier 2): the warp walks the
+// row once, each lane loading its 16-byte piece of x and of every router row
+// (two pieces of each in flight), exact products accumulated in fp64 (one
+// accumulator per row and per half of the unrolled pair), then the
+// butterfly.  Every term passes through at most H/32 + 6 roundings, inside
+// the H/32 + 16 of the tier-2 bound.
+__device__ void fp64_logits4(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* const (&w)[4], int nw,
+                             int H, double (&out)[4]) {
   const int lane = threadIdx.x & 31;
   const int vpr = H / 8;
-  double acc[4] = {0.0, 0.0, 0.0, 0.0};
   const uint4* xv = reinterpret_cast<const uint4*>(x);
-  const uint4* wv = reinterpret_cast<const uint4*>(w);
-  for (int c0 = lane; c0 < vpr; c0 += 128) {
-    uint4 xs[4], ws[4];
+  double acc[4][2] = {{0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}, {0.0, 0.0}};
+  for (int c0 = lane; c0 < vpr; c0 += 64) {
+    uint4 xs[2], ws[4][2];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int c = c0 + 32 * u;
       xs[u] = c < vpr ? xv[c] : make_uint4(0, 0, 0, 0);
-      ws[u] = c < vpr ? wv[c] : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        ws[r][u] = (r < nw && c < vpr) ? reinterpret_cast<const uint4*>(w[r])[c] : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float xf[8], wf[8];
+    for (int u = 0; u < 2; ++u) {
+      float xf[8];
       unpack8(xs[u], xf);
-      unpack8(ws[u], wf);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc[u] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[u]);
+      for (int r = 0; r < 4; ++r) {
+        float wf[8];
+        unpack8(ws[r][u], wf);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          acc[r][u] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[r][u]);
+      }
     }
   }
-  return warp_sum_d((acc[0] + acc[1]) + (acc[2] + acc[3]));
+#pragma unroll
+  for (int r = 0; r < 4; ++r) out[r] = warp_sum_d(acc[r][0] + acc[r][1]);
 }
 
 }  // namespace
@@ -524,7 +533,7 @@ __device__ void topk_token(
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
-    uint32_t* __restrict__ hdr) {
+    uint32_t* __restrict__ hdr, bool fp64_tier = false) {
   const int lane = threadIdx.x & 31;
   const int nper = (E + 31) / 32;
   float* row = logits + static_cast<size_t>(t) * E;
@@ -618,9 +627,12 @@ __device__ void topk_token(
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
   }
 
-  // certified when every adjacent gap among the top k+1 exceeds twice the bound
-  bool certified = true;
-  if (rmax > 0.f) {
+  // certified when every adjacent gap among the top k+1 exceeds twice the
+  // bound.  fp64_tier (logits from the tensor cores, whose bound is loose):
+  // every token goes to the fp64 tier, which also yields the weights.
+  bool certified = !fp64_tier;
+  double my_d = 0.0;   // fp64 logit of this lane's slot (tier 2)
+  if (certified && rmax > 0.f) {
     const double margin = 2.000001 * static_cast<double>(rmax);
     const float down = __shfl_down_sync(0xffffffffu, my_v, 1);
     const float next_v = lane == 31 ? extra_v : down;
@@ -633,11 +645,12 @@ __device__ void topk_token(
     if (lane == 0) atomicAdd(hdr + kHdrUncertain, 1u);
     const float kth_v = __shfl_sync(0xffffffffu, my_v, k - 1);
     int got = 0;
-    auto put = [&](int e) {   // slot `got` takes expert e
+    auto put = [&](int e, double d) {   // slot `got` takes expert e (fp64 logit d)
       if (lane == got) {
         my_idx = e;
         const float lv = __ldcg(row + e);
         my_v = isnan(lv) ? -FLT_MAX : lv;
+        my_d = d;
       }
       ++got;
     };
@@ -658,14 +671,21 @@ __device__ void topk_token(
     const double gamma64 = static_cast<double>(H / 32 + 16) * 1.1102230246251565e-16 * 1.0001;
     double r64 = 0.0;
     const __nv_bfloat16* xrow = hidden + static_cast<size_t>(t) * H;
-    for (int c = 0; c < nc; ++c) {
-      const int e = c_idx[c];
-      double d = fp64_logit(xrow, router_w + static_cast<size_t>(e) * H, H);
-      const double b = bias ? static_cast<double>(bias[e]) : 0.0;
-      d += b;
-      const double r = (gamma64 * xn * wnorm_of(e) + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
-      r64 = fmax(r64, r);
-      if (lane == 0) c_val[c] = d;
+    for (int c = 0; c < nc; c += 4) {   // four candidates per pass over the row
+      const int nw = min(4, nc - c);
+      const __nv_bfloat16* wrows[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) wrows[r] = router_w + static_cast<size_t>(c_idx[c + (r < nw ? r : 0)]) * H;
+      double dd[4];
+      fp64_logits4(xrow, wrows, nw, H, dd);
+      for (int r = 0; r < nw; ++r) {
+        const int e = c_idx[c + r];
+        const double b = bias ? static_cast<double>(bias[e]) : 0.0;
+        const double d = dd[r] + b;
+        const double rr = (gamma64 * xn * wnorm_of(e) + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
+        r64 = fmax(r64, rr);
+        if (lane == 0) c_val[c + r] = d;
+      }
     }
     __syncwarp();
     for (int c = lane; c < nc; c += 32) c_ord[c] = c;   // valid even if ranks collide (NaN)
@@ -689,7 +709,7 @@ __device__ void topk_token(
       int end = pos;
       while (end + 1 < nc && !(c_val[c_ord[end]] - c_val[c_ord[end + 1]] > margin64)) ++end;
       if (end == pos) {
-        put(c_idx[c_ord[pos]]);
+        put(c_idx[c_ord[pos]], c_val[c_ord[pos]]);
         pos = end + 1;
         continue;
       }
@@ -711,7 +731,7 @@ __device__ void topk_token(
             best_slot = m;
           }
         }
-        put(best_e);
+        put(best_e, c_val[c_ord[best_slot]]);
         __syncwarp();
         if (lane == 0) c_idx[c_ord[best_slot]] = -1;
         __syncwarp();
@@ -720,13 +740,36 @@ __device__ void topk_token(
     }
   }
 
-  // renormalised weights of the selected experts (fp32 softmax values)
-  const float p = lane < k ? expf(my_v - vmax) / se : 0.f;
+  // renormalised weights of the selected experts: fp32 softmax values
+  // renormalised over the k; on the fp64 tier the same quantity from the
+  // fp64 logits, exp(d_j - max_j d) / sum_j (the full softmax's denominator
+  // cancels in the renormalisation)
+  float p;
+  if (fp64_tier) {
+    double dm = lane < k ? my_d : -1.0e300;
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) dm = fmax(dm, __shfl_xor_sync(0xffffffffu, dm, m));
+    p = lane < k ? expf(static_cast<float>(my_d - dm)) : 0.f;
+  } else {
+    p = lane < k ? expf(my_v - vmax) / se : 0.f;
+  }
   const float psum = warp_sum(p);
   if (lane < k) {
     topk_ids[static_cast<size_t>(t) * k + lane] = my_idx;
     topk_w[static_cast<size_t>(t) * k + lane] = p / psum;
   }
+}
+
+// One warp per token.  With `with_align` (decode-sized calls) the CTA that
+// finishes last also runs the align: after a barrier (every top-k of the CTA
+// stored) its thread 0 takes an acquire-release ticket of the grid; the CTA
+// that draws the last one runs the align in its one-CTA form (its shared
+// memory holds the per-warp histograms).  No CTA waits for another; the
+// counter is reset by the CTA that completes it, so every call starts at 0.
+__device__ __forceinline__ unsigned int ticket_acq_rel(uint32_t* p) {
+  unsigned int old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
 }
 
 template <int kPer>
@@ -736,84 +779,25 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
-    uint32_t* __restrict__ hdr) {
-  pdl_wait();
-  pdl_launch_next();
-  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (t >= T) return;
-  topk_token<kPer>(t, logits, xnorm, wnorm, amax_tok, rsplit, nsplit, bias, hidden, router_w, T, H,
-                   E, k, gamma, ulast, topk_ids, topk_w, cand, hdr);
-}
-
-// ---------------------------------------------------------------------------
-// Fused decode router: logits, top-k and align in one launch, without
-// serialising the top-k of all tokens on one SM.  CTA (token tile, expert
-// group) computes its logits (every CTA also writes ||w_e|| of its experts,
-// identical values, so a token tile needs no other tile's CTAs); after a
-// barrier its thread 0 takes a ticket of the token tile (acquire-release at
-// GPU scope); the CTA that completes the tile runs the top-k of the tile's
-// tokens (one warp per token), then takes a ticket of the whole grid; the CTA
-// that completes the grid runs the align (the one-CTA form).  Tickets only:
-// no CTA ever waits for another, and each counter is reset by the CTA that
-// completes it, so every call starts from zero.  Used for decode-sized calls
-// (T*k < kAlignSliceMin, E <= 256, token tiles <= kRouterFusedMaxTiles).
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ unsigned int ticket_acq_rel(uint32_t* p) {
-  unsigned int old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
-  return old;
-}
-
-template <int TT, int ACC, int kPer>
-__global__ void __launch_bounds__(256) router_fused_kernel(RouterArgs ra, AlignArgs aa, float gamma,
-                                                           float ulast) {
-  extern __shared__ uint4 sx[];
+    uint32_t* __restrict__ hdr, AlignArgs aa, int with_align, int fp64_tier) {
+  extern __shared__ int align_hist[];
   __shared__ int s_last;
   pdl_wait();
   pdl_launch_next();
-  logits_body<TT, ACC>(ra.hidden, ra.router_w, ra.bias, ra.T, ra.H, ra.E, ra.logits, ra.xnorm, ra.wnorm,
-                       ra.amax_tok, sx, true);
-  __syncthreads();   // every logit, norm and amax of this CTA is stored
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t < T)
+    topk_token<kPer>(t, logits, xnorm, wnorm, amax_tok, rsplit, nsplit, bias, hidden, router_w, T, H,
+                     E, k, gamma, ulast, topk_ids, topk_w, cand, hdr, fp64_tier != 0);
+  if (!with_align) return;
+  __syncthreads();   // every top-k of this CTA is stored
   if (threadIdx.x == 0) {
-    uint32_t* cnt = ra.hdr + kHdrRouterTiles + blockIdx.x;
-    const bool last = ticket_acq_rel(cnt) == gridDim.y - 1;
-    if (last) *cnt = 0u;
-    s_last = last ? 1 : 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  // this CTA completes token tile blockIdx.x: top-k of its tokens
-  const int t0 = blockIdx.x * TT;
-  const int nt = min(TT, ra.T - t0);
-  for (int tt = threadIdx.x >> 5; tt < nt; tt += blockDim.x >> 5) {
-    const int t = t0 + tt;
-    topk_token<kPer>(t, ra.logits, ra.xnorm, ra.wnorm, ra.amax_tok, ra.rsplit, 1, ra.bias, ra.hidden,
-                     ra.router_w, ra.T, ra.H, ra.E, ra.k, gamma, ulast, ra.topk_ids, ra.topk_w, ra.cand, ra.hdr);
-  }
-  __syncthreads();   // every top-k of the tile is stored
-  if (threadIdx.x == 0) {
-    uint32_t* cnt = ra.hdr + kHdrRouterAll;
+    uint32_t* cnt = hdr + kHdrRouterAll;
     const bool last = ticket_acq_rel(cnt) == gridDim.x - 1;
     if (last) *cnt = 0u;
     s_last = last ? 1 : 0;
   }
   __syncthreads();
-  if (!s_last) return;
-  // this CTA completes the grid: the align, in the one-CTA form (the dynamic
-  // shared memory holds its per-warp histograms)
-  align_cta(aa, 0, 0, reinterpret_cast<int*>(sx));
-}
-
-template <int TT, int ACC, int kPer>
-static cudaError_t launch_fused(const RouterArgs& a, const AlignArgs& aa, float gamma, float ulast,
-                                cudaStream_t st) {
-  auto kern = router_fused_kernel<TT, ACC, kPer>;
-  const int hist = 8 * a.E * 4;
-  const int smem = TT * a.H * 2 > hist ? TT * a.H * 2 : hist;
-  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
-  if (err != cudaSuccess) return err;
-  dim3 grid((a.T + TT - 1) / TT, (a.E + 7) / 8);
-  return launch_pdl(kern, grid, dim3(256), smem, st, a, aa, gamma, ulast);
+  if (s_last) align_cta(aa, 0, 0, align_hist);
 }
 
 // ---------------------------------------------------------------------------
@@ -830,10 +814,16 @@ static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
 
 template <int kPer>
 static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, int nsplit,
-                               cudaStream_t st) {
-  return launch_pdl(router_topk_kernel<kPer>, dim3((a.T + 7) / 8), dim3(256), 0, st, a.logits,
-                    a.xnorm, a.wnorm, a.amax_tok, a.rsplit, nsplit, a.bias, a.hidden, a.router_w,
-                    a.T, a.H, a.E, a.k, gamma, ulast, a.topk_ids, a.topk_w, a.cand, a.hdr);
+                               cudaStream_t st, const AlignArgs* aa = nullptr, bool fp64_tier = false) {
+  const int smem = aa ? 8 * a.E * 4 : 0;   // the align's per-warp histograms (8 warps)
+  auto kern = router_topk_kernel<kPer>;
+  if (smem > 0) {
+    cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
+    if (err != cudaSuccess) return err;
+  }
+  return launch_pdl(kern, dim3((a.T + 7) / 8), dim3(256), smem, st, a.logits, a.xnorm, a.wnorm, a.amax_tok,
+                    a.rsplit, nsplit, a.bias, a.hidden, a.router_w, a.T, a.H, a.E, a.k, gamma, ulast,
+                    a.topk_ids, a.topk_w, a.cand, a.hdr, aa ? *aa : AlignArgs{}, aa ? 1 : 0, fp64_tier ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -919,10 +909,11 @@ static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStre
 }
 
 cudaError_t launch_router_topk(const RouterArgs& a, float gamma, float ulast, cudaStream_t st) {
-  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, 1, st);
-  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, 1, st);
-  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, 1, st);
-  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, 1, st);
+  // logits from the tensor cores: every token ranked and weighted on the fp64 tier
+  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, 1, st, nullptr, true);
+  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, 1, st, nullptr, true);
+  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, 1, st, nullptr, true);
+  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, 1, st, nullptr, true);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align, bool* fused) {
@@ -970,35 +961,6 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs*
         break;
       }
     }
-    // decode-sized calls: logits, top-k and align in one launch
-    const long long A = static_cast<long long>(a.T) * a.k;
-    const int tiles = (a.T + tt - 1) / tt;
-    if (fuse_align != nullptr && fused != nullptr && mode != kAcc32 && tt <= 4 && a.E <= 256 &&
-        A < kAlignSliceMin && tiles <= kRouterFusedMaxTiles && a.rsplit != nullptr) {
-      const int nchain_f = a.H / 32 + 16;
-      const double u32f = 5.9604644775390625e-08, u64f = 1.1102230246251565e-16;
-      const float gamma_f = mode == kAcc64 ? static_cast<float>(nchain_f * u64f * 1.0001)
-                                           : static_cast<float>((7.0 * u32f + nchain_f * u64f) * 1.0001);
-      const float ulast_f = static_cast<float>(u32f);
-      const int ecls = a.E <= 64 ? 0 : (a.E <= 128 ? 1 : 2);   // experts per lane 2, 4, 8
-      const int ti = tt == 1 ? 0 : (tt == 2 ? 1 : 2);
-      cudaError_t e2;
-      switch ((mode == kAcc64 ? 0 : 9) + 3 * ecls + ti) {
-#define MOE_FUSED_CASE(I, TT_, ACC_, KP_) \
-  case I: e2 = launch_fused<TT_, ACC_, KP_>(a, *fuse_align, gamma_f, ulast_f, st); break;
-        MOE_FUSED_CASE(0, 1, kAcc64, 2) MOE_FUSED_CASE(1, 2, kAcc64, 2) MOE_FUSED_CASE(2, 4, kAcc64, 2)
-        MOE_FUSED_CASE(3, 1, kAcc64, 4) MOE_FUSED_CASE(4, 2, kAcc64, 4) MOE_FUSED_CASE(5, 4, kAcc64, 4)
-        MOE_FUSED_CASE(6, 1, kAcc64, 8) MOE_FUSED_CASE(7, 2, kAcc64, 8) MOE_FUSED_CASE(8, 4, kAcc64, 8)
-        MOE_FUSED_CASE(9, 1, kAccMixed, 2) MOE_FUSED_CASE(10, 2, kAccMixed, 2) MOE_FUSED_CASE(11, 4, kAccMixed, 2)
-        MOE_FUSED_CASE(12, 1, kAccMixed, 4) MOE_FUSED_CASE(13, 2, kAccMixed, 4)
-        MOE_FUSED_CASE(14, 4, kAccMixed, 4) MOE_FUSED_CASE(15, 1, kAccMixed, 8)
-        MOE_FUSED_CASE(16, 2, kAccMixed, 8)
-        default: e2 = launch_fused<4, kAccMixed, 8>(a, *fuse_align, gamma_f, ulast_f, st); break;
-#undef MOE_FUSED_CASE
-      }
-      if (e2 == cudaSuccess) *fused = true;
-      return e2;
-    }
     switch (mode * 32 + tt) {
       case kAcc64 * 32 + 16: err = launch_logits<16, kAcc64>(a, st); break;
       case kAcc64 * 32 + 8: err = launch_logits<8, kAcc64>(a, st); break;
@@ -1027,10 +989,17 @@ cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs*
                       : mode == kAccMixed ? static_cast<float>((7.0 * u32 + nchain * u64) * 1.0001)
                                           : static_cast<float>(nchain * u32 * 1.0001);
   const float ulast = mode != kAcc32 ? static_cast<float>(u32) : static_cast<float>(2.0 * u32);
-  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, nsplit, st);
-  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, nsplit, st);
-  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, nsplit, st);
-  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, nsplit, st);
+  // decode-sized calls: the top-k kernel's last CTA also runs the align
+  const AlignArgs* aa = nullptr;
+  if (fuse_align != nullptr && fused != nullptr && a.E <= 256 &&
+      static_cast<long long>(a.T) * a.k < kAlignSliceMin) {
+    aa = fuse_align;
+    *fused = true;
+  }
+  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, nsplit, st, aa);
+  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, nsplit, st, aa);
+  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, nsplit, st, aa);
+  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, nsplit, st, aa);
 }
 
 }  // namespace moe
