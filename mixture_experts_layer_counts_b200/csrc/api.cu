@@ -376,8 +376,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     }
     if (any_normal) {
       GemmArgs g = g2;
-      g.chunks = at<int4>(ws, L.chunks_normal);
-      g.nchunks = hdr + kHdrChunksNormal;
+      g.chunks = at<int4>(ws, gemm_w2_pair() ? L.chunks_pair : L.chunks_normal);
+      g.nchunks = hdr + (gemm_w2_pair() ? kHdrChunksPair : kHdrChunksNormal);
       g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
       g.flags = flags + 3 * kMaxSlots;
       MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));

@@ -80,7 +80,8 @@ struct Cfg {
   static constexpr bool kDual = P == Proj::kW13;
   // normal-orientation gate/up GEMM: a unit is a 256-token chunk (two M
   // tiles) x one weight tile, so each weight byte staged feeds two MMAs
-  static constexpr bool kPair = !kSwap && kDual;
+  // gate/up always; down GEMM when launched with BNT == kPairTokens
+  static constexpr bool kPair = !kSwap && (kDual || BNT == kPairTokens);
   static constexpr int kChunkTokens = kPair ? kPairTokens : kNormalTokens;
   static constexpr int kBN = kSwap ? BNT : (kDual ? 128 : 256);   // max N
   static constexpr int kATile = kTileM * kAtomBytes;
@@ -372,7 +373,7 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
             mma_ss<FP8>(d0, sdesc_sw128(st + off), sdesc_sw128(st + C::kBOff + off), idesc, acc);
             if constexpr (C::kPair)
               if (ch.z > kTileM)
-                mma_ss<FP8>(d0 + 2 * C::kBN, sdesc_sw128(st + C::kATile + off),
+                mma_ss<FP8>(d0 + C::kNumAcc * C::kBN, sdesc_sw128(st + C::kATile + off),
                             sdesc_sw128(st + C::kBOff + off), idesc, acc);
           }
         }
@@ -624,6 +625,38 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
           }
           __syncwarp();
         }
+      } else if constexpr (C::kPair) {
+        // normal w2, 256-token chunk: warp half hx takes token rows
+        // hx*128 + q*32 + lane (M tile hx, whose accumulator sits at columns
+        // hx*kBN + [0, kBN)), all kBN columns, staged per warp like the w13
+        // epilogue; router-weighted fp32 rows to their slot rows f of ysc.
+        float* sw = epi + (warp - 2) * 32 * C::kEpiLd;
+        const int hx = (warp - 2) >> 2;
+        const int rb = hx * kTileM + q * 32;
+        const int f = rb + lane < nv ? a.perm[p0 + rb + lane] : -1;
+        const bool valid = f >= 0 && f < a.num_assign;
+        const float wt = valid ? a.topk_w[f] * scale : 0.f;
+        const int h0 = mt * C::kBN;
+        const uint32_t th = tbase + hx * C::kBN;
+        for (int c0 = 0; c0 < (rb < nv ? C::kBN : 0); c0 += C::kEpiCols) {
+          float v[16];
+          tmem_ld16_wait(th + c0, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<float4*>(sw + lane * C::kEpiLd + 4 * j) =
+                make_float4(v[4 * j] * wt, v[4 * j + 1] * wt, v[4 * j + 2] * wt, v[4 * j + 3] * wt);
+          __syncwarp();
+#pragma unroll
+          for (int r0 = 0; r0 < 32; r0 += 8) {
+            const int r = r0 + (lane >> 2);
+            const int fr = __shfl_sync(0xffffffffu, f, r);
+            const float4 val = *reinterpret_cast<const float4*>(sw + r * C::kEpiLd + 4 * (lane & 3));
+            if (fr >= 0 && fr < a.num_assign)
+              __stcs(reinterpret_cast<float4*>(static_cast<float*>(a.out) + static_cast<size_t>(fr) * a.ld_out +
+                                               h0 + c0 + 4 * (lane & 3)), val);
+          }
+          __syncwarp();
+        }
       } else {
         // normal w2: router-weighted fp32 rows of the unit's tokens, each to
         // its slot row f of ysc; warp half hx takes columns
@@ -727,8 +760,23 @@ cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tw, const
   if (p == Proj::kW13)
     return fp8 ? launch_one<Orient::kNormal, Proj::kW13, true, 1, 0>(tw, tx, a, grid, st)
                : launch_one<Orient::kNormal, Proj::kW13, false, 1, 0>(tw, tx, a, grid, st);
+  if (gemm_w2_pair())
+    return fp8 ? launch_one<Orient::kNormal, Proj::kW2, true, 1, kPairTokens>(tw, tx, a, grid, st)
+               : launch_one<Orient::kNormal, Proj::kW2, false, 1, kPairTokens>(tw, tx, a, grid, st);
   return fp8 ? launch_one<Orient::kNormal, Proj::kW2, true, 1, 0>(tw, tx, a, grid, st)
              : launch_one<Orient::kNormal, Proj::kW2, false, 1, 0>(tw, tx, a, grid, st);
+}
+
+// Normal-orientation down GEMM on 256-token chunks (two M tiles per staged
+// weight tile, 128 FLOP per staged byte) unless MOE_W2_PAIR=0 (128-token
+// tiles, two TMEM buffers; for measurements).
+bool gemm_w2_pair() {
+  static int v = -1;
+  if (v < 0) {
+    const char* s = std::getenv("MOE_W2_PAIR");
+    v = (s && std::atoi(s) == 0) ? 0 : 1;
+  }
+  return v == 1;
 }
 
 int gemm_token_box_rows(Orient o) { return o == Orient::kSwap ? kTokenBox : kNormalTokens; }

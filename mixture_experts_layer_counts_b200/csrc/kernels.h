@@ -167,6 +167,7 @@ enum class Orient { kSwap, kNormal };
 enum class Proj { kW13, kW2 };
 cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tm_w,
                         const CUtensorMap& tm_x, const GemmArgs& a, int grid, cudaStream_t st);
+bool gemm_w2_pair();                 // normal down GEMM on 256-token chunks (two M tiles)
 int gemm_token_box_rows(Orient o);   // rows per TMA box of the token operand
 int gemm_swap_chunk();               // largest token chunk of the swap-AB kernels
 int gemm_weight_box_rows(Orient o, Proj p);
