@@ -644,6 +644,33 @@ def sweep_orientation(local, counts=(8, 16, 24, 32, 48, 64, 80, 96, 128, 160, 19
         print(json.dumps(row), flush=True)
 
 
+def route_only(wl, local, steps=200):
+    """Device time of the router alone (moe_route: logits and top-k) on the
+    workload's hidden states and router weights; no expert weights are
+    allocated (small enough for full-set profiler captures).  One JSON line."""
+    from mixture_experts_layer_counts_b200 import layer
+    from mixture_experts_layer_counts_b200.inputs import make_hidden, make_router, zipf_bias
+
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    hidden, router_w = make_hidden(wl, dev), make_router(wl, dev)
+    bias = zipf_bias(wl["E"]).to(dev) if wl["zipf"] else None
+    ws = layer.make_workspace(wl["T"], wl["H"], wl["E"], 128, wl["top_k"], 0, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(5):
+        layer.moe_route(hidden, router_w, bias, wl["top_k"], workspace=ws)
+    ev = [new_events(2, stream) for _ in range(steps)]
+    torch.cuda.synchronize()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        layer.moe_route(hidden, router_w, bias, wl["top_k"], workspace=ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    us = 1e3 * statistics.median(a.elapsed_time(b) for a, b in ev)
+    print(json.dumps({"route_only": describe(wl), "us": us, "steps": steps}), flush=True)
+
+
 def run_ours(args, wl, rank, world, local):
     pk = peaks()
     head, cpu = measure_workload(args.workload, wl, args, rank, world, local, steps_exact=args.steps)
@@ -691,6 +718,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only-headline", action="store_true", help="skip the other workloads")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time the router alone on the workload's hidden states (no expert weights)")
     ap.add_argument("--sweep-orientation", action="store_true",
                     help="time both GEMMs under forced swap-AB / normal orientation over tokens per expert")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -721,6 +750,9 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     if args.sweep_orientation:
         sweep_orientation(local)
+        return
+    if args.route_only:
+        route_only(wl, local, args.steps)
         return
     try:
         run_ours(args, wl, rank, world, local)
