@@ -12,7 +12,26 @@
 //   in fp32, each product and each sum rounded separately (no fused
 //   multiply-add); scale = fp32(amax|y|) / 448 (amax 0 -> 1); code =
 //   E4M3(fp32(y / scale)), round-to-nearest-even, saturating to +-448.
-//   A position outside [0, max_pos) yields codes 0 and scale 0.
+//   A position outside [0, max_pos) yields codes 0 and scale 0.  Inputs are
+//   finite (a NaN or an infinity in x gives unspecified codes and scale).
+//
+// The division without a divide.  The kernel is bound by instruction issue,
+// not by HBM, and a correctly rounded fp32 division costs about ten
+// instructions per element.  Markstein's theorem (P. Markstein, "Computation
+// of elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+// Dev. 34(1), 1990; also the Handbook of Floating-Point Arithmetic, division
+// with a fused multiply-add) gives the same result in three: with r the
+// correctly rounded 1/s and q0 = RN(y r) (within one ulp of y/s), the
+// residual e = y - q0 s is exact in one FMA and RN(q0 + e r) is the correctly
+// rounded y/s, barring underflow and overflow (checked per head: the divide
+// serves scales outside [2^-100, 2^100]).  The kernel runs it on negated
+// values, n0 = RN(y * -r), e = RN(n0 s + y), n1 = RN(e * -r + n0) = -RN(y/s),
+// which also gives a zero quotient the sign of y (the plain order turns -0
+// into +0); the codes of the negated quotients are flipped back with one XOR
+// per four codes (E4M3 is sign-magnitude and its rounding symmetric).  The
+// two lanes of each step share one packed fp32x2 instruction (sm_100).  The
+// rotation stays in scalar multiplies and adds with explicit rounding, so no
+// product is fused into the sum.
 //
 // Layout and work split.  x [T, nH, D] bf16, codes [T, nH, D] E4M3, scales
 // [T, nH] fp32, tables [max_pos, D/2] fp32.  A head's D/2 pairs are covered by
@@ -20,8 +39,11 @@
 // bytes of each table row, 8 bytes of codes per half.  A warp takes 512/D
 // consecutive heads (the lanes of a head reduce their amax with shuffles), the
 // grid strides over the heads, so loads and stores are contiguous 16-byte
-// vectors.  HBM-bound: per head 2 D bytes of x read, D bytes of codes and 4
-// bytes of scale written (the table rows are shared by a token's heads).
+// vectors.  The roofline is HBM: per head 2 D bytes of x read, D bytes of
+// codes and 4 bytes of scale written (the table rows are shared by a token's
+// heads); the kernel runs at about half of it, bound by instruction issue, and
+// is held to 40 registers (six CTAs per SM), which outruns the unbounded
+// 55-register build despite a few spilled values.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -38,6 +60,23 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
+// Packed fp32x2 multiply and fused multiply-add, round-to-nearest-even (lane x in the low half).
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
 __device__ __forceinline__ void bf16x8(const uint4& v, float (&f)[8]) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -50,7 +89,7 @@ __device__ __forceinline__ void bf16x8(const uint4& v, float (&f)[8]) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) inv_rope_fp8_kernel(
+__global__ void __launch_bounds__(256, 6) inv_rope_fp8_kernel(
     const uint4* __restrict__ x, const int32_t* __restrict__ pos, const float4* __restrict__ cos_tab,
     const float4* __restrict__ sin_tab, long long n_heads_total, int nH, int D, int max_pos,
     uint2* __restrict__ codes, float* __restrict__ scales) {
@@ -94,13 +133,30 @@ __global__ void __launch_bounds__(256) inv_rope_fp8_kernel(
     uint2 qa = make_uint2(0u, 0u), qb = make_uint2(0u, 0u);
     if (valid) {
       float d0[8], d1[8];
+      if (scale >= 0x1p-100f && scale <= 0x1p100f) {
+        const float nr = -__frcp_rn(scale);
+        const float2 NR = make_float2(nr, nr), SC = make_float2(scale, scale);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        d0[i] = __fdiv_rn(y0[i], scale);
-        d1[i] = __fdiv_rn(y1[i], scale);
+        for (int i = 0; i < 8; i += 2) {
+          const float2 Y0 = make_float2(y0[i], y0[i + 1]), Y1 = make_float2(y1[i], y1[i + 1]);
+          const float2 n0 = mul2(Y0, NR), n1 = mul2(Y1, NR);
+          const float2 e0 = fma2(n0, SC, Y0), e1 = fma2(n1, SC, Y1);
+          const float2 q0 = fma2(e0, NR, n0), q1 = fma2(e1, NR, n1);
+          d0[i] = q0.x; d0[i + 1] = q0.y; d1[i] = q1.x; d1[i + 1] = q1.y;
+        }
+        qa = make_uint2(e4m3x4(d0[0], d0[1], d0[2], d0[3]) ^ 0x80808080u,
+                        e4m3x4(d0[4], d0[5], d0[6], d0[7]) ^ 0x80808080u);
+        qb = make_uint2(e4m3x4(d1[0], d1[1], d1[2], d1[3]) ^ 0x80808080u,
+                        e4m3x4(d1[4], d1[5], d1[6], d1[7]) ^ 0x80808080u);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          d0[i] = __fdiv_rn(y0[i], scale);
+          d1[i] = __fdiv_rn(y1[i], scale);
+        }
+        qa = make_uint2(e4m3x4(d0[0], d0[1], d0[2], d0[3]), e4m3x4(d0[4], d0[5], d0[6], d0[7]));
+        qb = make_uint2(e4m3x4(d1[0], d1[1], d1[2], d1[3]), e4m3x4(d1[4], d1[5], d1[6], d1[7]));
       }
-      qa = make_uint2(e4m3x4(d0[0], d0[1], d0[2], d0[3]), e4m3x4(d0[4], d0[5], d0[6], d0[7]));
-      qb = make_uint2(e4m3x4(d1[0], d1[1], d1[2], d1[3]), e4m3x4(d1[4], d1[5], d1[6], d1[7]));
     }
     codes[hd * (2 * half_v) + q] = qa;
     codes[hd * (2 * half_v) + half_v + q] = qb;

@@ -54,3 +54,45 @@ def test_inv_rope_fp8_large_call_sampled(cuda_ok):
     rng = np.random.default_rng(0)
     sample = np.sort(np.concatenate([[0, 1, 2, T - 1], rng.choice(np.arange(3, T - 1), 60, replace=False)]))
     run_case(T, 32, 128, 8192, seed=7, sample=sample)
+
+
+def e4m3_midpoints():
+    """Every midpoint between neighbouring positive E4M3 values (the ties of
+    its round-to-nearest-even)."""
+    vals = sorted({(1 + m / 8) * 2.0 ** (e - 7) for e in range(1, 16) for m in range(8)} |
+                  {m / 8 * 2.0 ** -6 for m in range(1, 8)})
+    vals = [v for v in vals if v <= 448]
+    mids = [(a + b) / 2 for a, b in zip(vals, vals[1:])]
+    return np.array(mids)
+
+
+def test_inv_rope_fp8_rounding_boundaries(cuda_ok):
+    """Quotients exactly on (and next to) E4M3 ties, under scales whose
+    reciprocal is inexact, and heads so small that the scale is subnormal
+    (no finite reciprocal): the kernel's reciprocal path must fall back to the
+    division wherever that decides the code.  Position 0 (cos 1, sin 0) keeps
+    y = x exactly, so the ties reach the quantiser intact."""
+    T, nH, D = 48, 4, 128
+    rng = np.random.default_rng(11)
+    mids = e4m3_midpoints()
+    ks = [1.0, 3.0, 5.0, 7.0, 0.75, 3.0 * 2 ** -20, 5.0 * 2 ** 20]
+    x = np.zeros((T, nH, D))
+    for t in range(T):
+        for h in range(nH):
+            k = ks[(t * nH + h) % len(ks)]
+            if (t * nH + h) % 11 == 10:
+                k = 2.0 ** -rng.integers(128, 140)               # subnormal scale
+            row = k * rng.choice(mids, D) * rng.choice([-1.0, 1.0], D)
+            row[rng.integers(D)] = 448.0 * k * rng.choice([-1.0, 1.0])
+            x[t, h] = row
+    xt = torch.tensor(x, dtype=torch.float32).to(torch.bfloat16)
+    exact = (xt.double().numpy() == x)
+    assert exact.mean() > 0.8, "too few engineered values survive the bf16 cast"
+    ct, st = tables(16, D // 2)
+    pos = np.zeros(T, dtype=np.int32)
+    codes, scales = layer.inv_rope_fp8_quant(xt.cuda(), torch.from_numpy(pos).cuda(), torch.from_numpy(ct).cuda(),
+                                             torch.from_numpy(st).cuda())
+    torch.cuda.synchronize()
+    rc, rs = inv_rope_fp8_ref(xt.float().numpy(), pos, ct, st)
+    assert np.array_equal(scales.cpu().numpy(), rs), "scales differ"
+    assert np.array_equal(codes.cpu().numpy(), rc), "codes differ"
