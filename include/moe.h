@@ -111,9 +111,9 @@ typedef struct {
  * activations, the intermediate and the per-slot fp32 down-projection rows. */
 size_t moe_workspace_size(int T, int H, int E, int I, int top_k, int dtype);
 
-/* Zero the workspace's header (its first 256 bytes: the status words and a
- * counter that every call leaves at zero again).  Call once on a fresh
- * workspace before its first use. */
+/* Zero the workspace's header (its first 1024 bytes: the status words and the
+ * counters and flags that every call leaves at zero again).  Call once on a
+ * fresh workspace before its first use, and again after a call that failed. */
 moe_status_t moe_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* The whole layer.

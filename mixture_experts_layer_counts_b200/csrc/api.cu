@@ -173,11 +173,28 @@ void record(moe_debug_out_t* dbg, int i, cudaStream_t st) {
 // the last place of the running magnitude per instruction (H / 16
 // instructions; a factor 2 of margin).  Tokens whose top-(k+1) gaps that
 // bound cannot separate are re-ranked in fp64, then exactly, as on every path.
+// Router path: logits on the tensor cores (route_tc) once the logit work
+// passes 2^28 multiply-adds (large batches, where the CUDA-core kernels are
+// bound by their arithmetic), else the CUDA-core logits kernels, whose
+// tighter bounds certify most tokens without a second pass.  MOE_ROUTER=tc or
+// =simt fixes the path for calls that need not be batch-invariant (for
+// measurements and tests).
 bool tc_router_eligible(int T, int H, int E, bool invariant) {
-  return !invariant && static_cast<double>(T) * E * H > static_cast<double>(1 << 28);
+  static int force = -1;   // 0: size rule, 1: tensor cores, 2: CUDA cores
+  if (force < 0) {
+    const char* s = std::getenv("MOE_ROUTER");
+    force = !s ? 0 : (std::strcmp(s, "tc") == 0 ? 1 : (std::strcmp(s, "simt") == 0 ? 2 : 0));
+  }
+  if (invariant || force == 2) return false;
+  return force == 1 || static_cast<double>(T) * E * H > static_cast<double>(1 << 28);
 }
 
-moe_status_t route_tc(const RouterArgs& ra, int grid, unsigned long long timeout_ns, cudaStream_t st) {
+// Logits on the tensor cores as a dense swap-AB GEMM (router rows = M, tokens
+// = N), its K loop split over the grid with partial tiles when `ra.partials`
+// is given (flags in the workspace header, cleared again by their consumer),
+// then the candidate re-evaluation top-k (launch_router_topk_tc).
+moe_status_t route_tc(const RouterArgs& ra, int grid, unsigned long long timeout_ns, cudaStream_t st,
+                      const AlignArgs* fuse_align = nullptr, bool* fused = nullptr) {
   CUtensorMap tw, tx;
   MOE_TRY(make_tmap(&tw, ra.router_w, false, ra.H, ra.E, gemm_weight_box_rows(Orient::kSwap, Proj::kW2)));
   MOE_TRY(make_tmap(&tx, ra.hidden, false, ra.H, ra.T, gemm_token_box_rows(Orient::kSwap)));
@@ -200,11 +217,16 @@ moe_status_t route_tc(const RouterArgs& ra, int grid, unsigned long long timeout
   g.num_assign = ra.T;
   g.hdr = ra.hdr;
   g.timeout_ns = timeout_ns;
-  g.whole_units = 1;
+  g.whole_units = ra.partials != nullptr ? 0 : 1;
+  g.partials = ra.partials;
+  g.flags = reinterpret_cast<int*>(ra.hdr + kHdrRouterFlags);
+  g.flags_self_reset = 1;
   MOE_TRY(cuda_status(launch_gemm(Orient::kSwap, Proj::kW2, false, tw, tx, g, grid, st)));
-  const float gamma = static_cast<float>(static_cast<double>(ra.H) * 2.384185791015625e-07);   // H * 2^-22
-  const float ulast = 5.9604644775390625e-08f;                                                 // the bias add
-  return cuda_status(launch_router_topk(ra, gamma, ulast, st));
+  // H 2^-22 ||x|| ||w||: the tensor-core accumulation order and rounding are
+  // not specified, so the bound allows four ulps of sum|x w| per product
+  const float gamma = static_cast<float>(static_cast<double>(ra.H) * 2.384185791015625e-07);
+  const float ulast = 1.1920928955078125e-07f;   // the partial-tile adds, the bias add
+  return cuda_status(launch_router_topk_tc(ra, gamma, ulast, st, fuse_align, fused));
 }
 
 moe_status_t forward_impl(const void* hidden, const void* router_w, const float* router_bias,
@@ -257,7 +279,8 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                 router_bias, T, H, E, k,
                 at<float>(ws, L.logits), at<float>(ws, L.xnorm), at<float>(ws, L.wnorm),
                 at<float>(ws, L.amax_tok), at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_w),
-                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0};
+                at<unsigned char>(ws, L.cand), hdr, at<float>(ws, L.rsplit), invariant ? 1 : 0,
+                at<float>(ws, L.partials)};
   AlignArgs aa{at<int32_t>(ws, L.topk_ids), T, E, k,
                at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets), at<int32_t>(ws, L.perm),
                at<int32_t>(ws, L.inv_perm), at<int4>(ws, L.chunks_swap), at<int4>(ws, L.chunks_normal),
@@ -272,7 +295,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
                                             ? static_cast<unsigned long long>(dbg->wait_timeout_us) * 1000ull
                                             : kWaitTimeoutNs;
   if (tc_router_eligible(T, H, E, invariant))
-    MOE_TRY(route_tc(ra, grid, timeout_ns, st));
+    MOE_TRY(route_tc(ra, grid, timeout_ns, st, &aa, &fused_route));
   else
     MOE_TRY(cuda_status(launch_router(ra, st, invariant ? nullptr : &aa, &fused_route)));
   record(dbg, 1, st);
@@ -671,7 +694,7 @@ moe_status_t moe_route(const void* hidden, const void* router_w, const float* ro
                 at<float>(workspace, L.logits), at<float>(workspace, L.xnorm),
                 at<float>(workspace, L.wnorm), at<float>(workspace, L.amax_tok), topk_ids, topk_w,
                 at<unsigned char>(workspace, L.cand), at<uint32_t>(workspace, L.header),
-                at<float>(workspace, L.rsplit)};
+                at<float>(workspace, L.rsplit), 0, at<float>(workspace, L.partials)};
   if (tc_router_eligible(T, H, E, false)) {
     const int grid = device_sm_count() < kMaxSlots ? device_sm_count() : kMaxSlots;
     return route_tc(ra, grid, kWaitTimeoutNs, static_cast<cudaStream_t>(stream));

@@ -53,7 +53,9 @@ constexpr int kHdrScaleS2 = 9;         // fp32 bits: intermediate scale (FP8)
 constexpr int kHdrBarrier = 12;        // grid barrier counter
 constexpr int kHdrRouterAll = 13;      // top-k CTAs finished (decode calls: the last one aligns;
                                        // reset by that CTA, so every call starts at 0)
-constexpr int kHeaderBytes = 256;
+constexpr int kHdrRouterFlags = 64;    // words 64 .. 64 + kMaxSlots - 1: split-unit flags of the
+                                       // tensor-core router GEMM (zeroed again by their consumer)
+constexpr int kHeaderBytes = 1024;
 constexpr int kStatusBytes = kHeaderBytes;
 
 __device__ __forceinline__ void report_status(uint32_t* status, uint32_t code, uint32_t where) {

@@ -399,23 +399,35 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     int it = 0;
     if (a.dense_T > 0 && a.xnorm != nullptr) {
       // router logits: while the first tiles stream in, these warps write the
-      // norms and amax of a grid-strided share of the token and router rows
+      // norms (and amax) of a share of the router rows and, when norm_x is
+      // given, of the token rows, strided over the active CTAs (0 .. nact-1;
+      // the others run no epilogue)
       const int vpr = a.norm_H / 8;
       const long long rows = static_cast<long long>(a.dense_T) + a.n_cols;
-      for (long long r = static_cast<long long>(blockIdx.x) * C::kEpiWarps + (warp - 2); r < rows;
-           r += static_cast<long long>(gridDim.x) * C::kEpiWarps) {
+      const long long first = a.norm_x != nullptr ? 0 : a.dense_T;
+      const long long nact = rr ? (nunits < gridDim.x ? nunits : static_cast<long long>(gridDim.x)) : G;
+      for (long long r = first + static_cast<long long>(blockIdx.x) * C::kEpiWarps + (warp - 2); r < rows;
+           r += nact * C::kEpiWarps) {
         const bool tok = r < a.dense_T;
         const uint4* src = static_cast<const uint4*>(tok ? a.norm_x : a.norm_w) +
                            static_cast<size_t>(tok ? r : r - a.dense_T) * vpr;
         float ss = 0.f, am = 0.f;
-        for (int c = lane; c < vpr; c += 32) {
-          const uint4 v4 = src[c];
-          const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4);
+        for (int c0 = lane; c0 < vpr; c0 += 32 * 8) {   // eight 16-byte loads in flight per lane
+          uint4 v4[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float2 f2 = __bfloat1622float2(b2[i]);
-            ss = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, ss));
-            am = fmaxf(am, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+          for (int u = 0; u < 8; ++u) {
+            const int c = c0 + 32 * u;
+            v4[u] = c < vpr ? src[c] : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&v4[u]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f2 = __bfloat1622float2(b2[i]);
+              ss = fmaf(f2.x, f2.x, fmaf(f2.y, f2.y, ss));
+              am = fmaxf(am, fmaxf(fabsf(f2.x), fabsf(f2.y)));
+            }
           }
         }
 #pragma unroll
@@ -713,6 +725,18 @@ __global__ void __launch_bounds__((Cfg<O, P, FP8, KA, BNT>::kThreads), 1)
     }
   }
   if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (a.flags_self_reset && !rr && threadIdx.x == 0 && active && my_a1 > my_a0) {
+    // Flags that no later kernel clears: only the last unit of this CTA's
+    // range can continue on later CTAs, whose flags this CTA consumed (or
+    // gave up on, which leaves the call failed and the workspace to be
+    // initialised again).  Each of those CTAs sets its flag once per launch.
+    const long long u_last = (my_a1 - 1) / ksteps;
+    const long long u_begin = u_last * ksteps, u_end = u_begin + ksteps;
+    if (u_begin >= my_a0 && u_end > my_a1) {
+      const int last = atom_owner(u_end - 1, W, G);
+      for (int c2 = blockIdx.x + 1; c2 <= last; ++c2) a.flags[c2] = 0;
+    }
+  }
   if constexpr (FP8 && C::kDual) {
     if (a.amax_n > 0) requant_tail(a, red, abort_flag);   // red / abort_flag reused as smem words
   }

@@ -59,16 +59,21 @@ struct RouterArgs {
   uint32_t* hdr;
   float* rsplit;          // router_split_floats(T, E) floats, or NULL (no split-K)
   int invariant;          // 1: one logits kernel and summation order for every T (no split-K)
+  float* partials;        // GEMM partial tiles for the tensor-core logits (NULL: whole units)
 };
 struct AlignArgs;
 // fuse_align non-NULL: a decode-sized call may run logits, top-k and align in
 // one launch (then *fused is set and the align must not be launched again).
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align = nullptr,
                           bool* fused = nullptr);
-// The router's top-k kernel alone (logits, norms and amax already written),
-// with the relative error bound `gamma` of the logits (times ||x|| ||w||) and
-// `ulast` of their last roundings.
-cudaError_t launch_router_topk(const RouterArgs& a, float gamma, float ulast, cudaStream_t st);
+// The top-k of logits from the tensor cores (logits, norms and amax already
+// written), with the relative error bound `gamma` of the logits (times
+// ||x|| ||w||) and `ulast` of their last roundings: one warp per token, every
+// candidate within twice the bound of the k-th re-evaluated in mixed
+// precision (in fp64 where that leaves the order open).  With
+// `aa` non-NULL a decode-sized call's last CTA also runs the align (*fused set).
+cudaError_t launch_router_topk_tc(const RouterArgs& a, float gamma, float ulast, cudaStream_t st,
+                                  const AlignArgs* aa = nullptr, bool* fused = nullptr);
 
 struct AlignArgs {
   const int32_t* topk_ids;
@@ -133,6 +138,8 @@ struct GemmArgs {
   uint32_t* hdr;
   float* partials;             // kMaxSlots fp32 partial tiles (split units)
   int* flags;                  // kMaxSlots flags, zero at launch
+  int flags_self_reset;        // 1: the CTA that consumes a split unit's flags zeroes them again
+                               // (flags that no align kernel clears, e.g. the router's)
   unsigned long long timeout_ns;   // limit of every bounded wait in the kernel
   int inject_stall;            // failure-path test: CTA 0 leaves one stage unfilled
   // Router logits mode of the swap-AB down-projection kernel (dense_T > 0):

@@ -17,6 +17,13 @@
 //      their exact values, accumulated as 640-bit fixed-point integers.
 // Softmax and the renormalised weights are computed in fp32 from the fp32
 // logits, one warp per token with shuffle reductions.
+// Large batches take their logits from the tensor cores instead (a dense
+// swap-AB GEMM of the grouped-GEMM kernel).  Their bound is loose (the
+// accumulation order and rounding inside the MMA are not specified), so every
+// token goes through tier 2 for its candidates, first in mixed precision (fp32
+// blocks of 8 products, fp64 sums: a bound of about 7 fp32 ulps of sum|x w|),
+// then in fp64 when that leaves a gap open; the weights come from those
+// re-evaluated logits.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -141,14 +148,20 @@ __device__ __forceinline__ int exact_cmp(const long long (&a)[kLimbs], const lon
   return 0;
 }
 
-// Up to four fp64 logits of one token row at once (tier 2): the warp walks the
+// Up to four logits of one token row at once (tier 2): the warp walks the
 // row once, each lane loading its 16-byte piece of x and of every router row
-// (two pieces of each in flight), exact products accumulated in fp64 (one
-// accumulator per row and per half of the unrolled pair), then the
-// butterfly.  Every term passes through at most H/32 + 6 roundings, inside
-// the H/32 + 16 of the tier-2 bound.
-__device__ void fp64_logits4(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* const (&w)[4], int nw,
-                             int H, double (&out)[4]) {
+// (two pieces of each in flight), exact products accumulated with one
+// accumulator per row and per half of the unrolled pair, then the butterfly.
+// kMixed = false: every product added in fp64; each term passes through at
+// most H/32 + 6 roundings, inside the H/32 + 16 of the fp64 bound.
+// kMixed = true: the 8 products of each 16-byte vector pair summed by an fp32
+// FMA chain (7 roundings), the vector sums added in fp64: one fp64
+// conversion per 8 products instead of two per product; error at most
+// (7 u32 + (H/256 + 16) u64) sum|x w| (1 + 1e-4), plus H 2^-148 for values
+// below fp32's normal range.
+template <bool kMixed>
+__device__ void logits4(const __nv_bfloat16* __restrict__ x, const __nv_bfloat16* const (&w)[4], int nw,
+                        int H, double (&out)[4]) {
   const int lane = threadIdx.x & 31;
   const int vpr = H / 8;
   const uint4* xv = reinterpret_cast<const uint4*>(x);
@@ -171,14 +184,87 @@ __device__ void fp64_logits4(const __nv_bfloat16* __restrict__ x, const __nv_bfl
       for (int r = 0; r < 4; ++r) {
         float wf[8];
         unpack8(ws[r][u], wf);
+        if constexpr (kMixed) {
+          float p = xf[0] * wf[0];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          acc[r][u] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[r][u]);
+          for (int i = 1; i < 8; ++i) p = fmaf(xf[i], wf[i], p);
+          acc[r][u] += static_cast<double>(p);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            acc[r][u] = fma(static_cast<double>(xf[i]), static_cast<double>(wf[i]), acc[r][u]);
+        }
       }
     }
   }
 #pragma unroll
   for (int r = 0; r < 4; ++r) out[r] = warp_sum_d(acc[r][0] + acc[r][1]);
+}
+
+// Rank the nc candidates (c_idx, c_val) by (value desc, index asc) into
+// c_ord (c_ord[rank] = candidate slot), by the calling warp.
+__device__ void rank_candidates(const int* c_idx, int* c_ord, const double* c_val, int nc) {
+  const int lane = threadIdx.x & 31;
+  for (int c = lane; c < nc; c += 32) c_ord[c] = c;   // valid even if ranks collide (NaN)
+  __syncwarp();
+  for (int c = lane; c < nc; c += 32) {
+    const double vc = c_val[c];
+    const int ic = c_idx[c];
+    int rank = 0;
+    for (int j = 0; j < nc; ++j) {
+      const double vj = c_val[j];
+      rank += (vj > vc || (vj == vc && c_idx[j] < ic)) ? 1 : 0;
+    }
+    if (rank < nc) c_ord[rank] = c;
+  }
+  __syncwarp();
+}
+
+// The k selected experts in order, from ranked candidates whose values carry
+// errors below margin / 2 (by the calling warp).  Runs of candidates closer
+// than `margin` are ordered by their exact values (tier 3); put(e, d) takes
+// them in order.  Marks chosen candidates with c_idx = -1.
+template <typename Put>
+__device__ void assemble_in_order(int* c_idx, const int* c_ord, const double* c_val, int nc, int k,
+                                  double margin, const __nv_bfloat16* __restrict__ xrow,
+                                  const __nv_bfloat16* __restrict__ router_w, const float* __restrict__ bias,
+                                  int H, int& got, Put&& put) {
+  const int lane = threadIdx.x & 31;
+  int pos = 0;
+  const uint16_t* xbits = reinterpret_cast<const uint16_t*>(xrow);
+  while (got < k && pos < nc) {
+    int end = pos;
+    while (end + 1 < nc && !(c_val[c_ord[end]] - c_val[c_ord[end + 1]] > margin)) ++end;
+    if (end == pos) {
+      put(c_idx[c_ord[pos]], c_val[c_ord[pos]]);
+      pos = end + 1;
+      continue;
+    }
+    const int need = min(end - pos + 1, k - got);
+    for (int q = 0; q < need; ++q) {
+      long long best[kLimbs];
+      int best_e = -1, best_slot = -1;
+      for (int m = pos; m <= end; ++m) {
+        const int e = c_idx[c_ord[m]];
+        if (e < 0) continue;   // already chosen
+        long long cur[kLimbs];
+        exact_logit(xbits, reinterpret_cast<const uint16_t*>(router_w) + static_cast<size_t>(e) * H,
+                    bias ? bias[e] : 0.f, H, cur);
+        int cmp = best_e < 0 ? 1 : exact_cmp(cur, best);
+        if (cmp > 0 || (cmp == 0 && e < best_e)) {
+#pragma unroll
+          for (int i = 0; i < kLimbs; ++i) best[i] = cur[i];
+          best_e = e;
+          best_slot = m;
+        }
+      }
+      put(best_e, c_val[c_ord[best_slot]]);
+      __syncwarp();
+      if (lane == 0) c_idx[c_ord[best_slot]] = -1;
+      __syncwarp();
+    }
+    pos = end + 1;
+  }
 }
 
 }  // namespace
@@ -533,7 +619,7 @@ __device__ void topk_token(
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
-    uint32_t* __restrict__ hdr, bool fp64_tier = false) {
+    uint32_t* __restrict__ hdr, bool tc_tier) {
   const int lane = threadIdx.x & 31;
   const int nper = (E + 31) / 32;
   float* row = logits + static_cast<size_t>(t) * E;
@@ -628,10 +714,10 @@ __device__ void topk_token(
   }
 
   // certified when every adjacent gap among the top k+1 exceeds twice the
-  // bound.  fp64_tier (logits from the tensor cores, whose bound is loose):
-  // every token goes to the fp64 tier, which also yields the weights.
-  bool certified = !fp64_tier;
-  double my_d = 0.0;   // fp64 logit of this lane's slot (tier 2)
+  // bound.  tc_tier (logits from the tensor cores, whose bound is loose):
+  // every token re-evaluates its candidates, which also yields the weights.
+  bool certified = !tc_tier;
+  double my_d = 0.0;   // re-evaluated logit of this lane's slot (tc_tier)
   if (certified && rmax > 0.f) {
     const double margin = 2.000001 * static_cast<double>(rmax);
     const float down = __shfl_down_sync(0xffffffffu, my_v, 1);
@@ -642,10 +728,12 @@ __device__ void topk_token(
   }
 
   if (!certified) {
-    if (lane == 0) atomicAdd(hdr + kHdrUncertain, 1u);
+    // counted here for CUDA-core logits; from tensor-core logits every token
+    // comes here, and only the ones the mixed values leave open are counted
+    if (lane == 0 && !tc_tier) atomicAdd(hdr + kHdrUncertain, 1u);
     const float kth_v = __shfl_sync(0xffffffffu, my_v, k - 1);
     int got = 0;
-    auto put = [&](int e, double d) {   // slot `got` takes expert e (fp64 logit d)
+    auto put = [&](int e, double d) {   // slot `got` takes expert e (re-evaluated logit d)
       if (lane == got) {
         my_idx = e;
         const float lv = __ldcg(row + e);
@@ -654,7 +742,7 @@ __device__ void topk_token(
       }
       ++got;
     };
-    // ---- tier 2: candidates re-evaluated in fp64 --------------------------
+    // ---- tier 2: candidates re-evaluated on the CUDA cores ----------------
     int* c_idx = reinterpret_cast<int*>(cand + static_cast<size_t>(t) * E * 16);
     int* c_ord = c_idx + E;
     double* c_val = reinterpret_cast<double*>(c_ord + E);
@@ -668,84 +756,58 @@ __device__ void topk_token(
       nc += __popc(bal);
     }
     __syncwarp();
-    const double gamma64 = static_cast<double>(H / 32 + 16) * 1.1102230246251565e-16 * 1.0001;
-    double r64 = 0.0;
+    const double u32 = 5.9604644775390625e-08, u64 = 1.1102230246251565e-16;
     const __nv_bfloat16* xrow = hidden + static_cast<size_t>(t) * H;
-    for (int c = 0; c < nc; c += 4) {   // four candidates per pass over the row
-      const int nw = min(4, nc - c);
-      const __nv_bfloat16* wrows[4];
+    // every candidate's logit (+ bias) into c_val, ranked; returns the largest bound
+    auto evaluate = [&](bool mixed) -> double {
+      const double g = mixed ? (7.0 * u32 + (H / 256 + 16) * u64) * 1.0001
+                             : static_cast<double>(H / 32 + 16) * u64 * 1.0001;
+      const double floor_err = mixed ? static_cast<double>(H) * 3.5032461608120427e-45 : 1e-300;
+      double rmx = 0.0;
+      for (int c = 0; c < nc; c += 4) {   // four candidates per pass over the row
+        const int nw = min(4, nc - c);
+        const __nv_bfloat16* wrows[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) wrows[r] = router_w + static_cast<size_t>(c_idx[c + (r < nw ? r : 0)]) * H;
-      double dd[4];
-      fp64_logits4(xrow, wrows, nw, H, dd);
-      for (int r = 0; r < nw; ++r) {
-        const int e = c_idx[c + r];
-        const double b = bias ? static_cast<double>(bias[e]) : 0.0;
-        const double d = dd[r] + b;
-        const double rr = (gamma64 * xn * wnorm_of(e) + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + 1e-300;
-        r64 = fmax(r64, rr);
-        if (lane == 0) c_val[c + r] = d;
-      }
-    }
-    __syncwarp();
-    for (int c = lane; c < nc; c += 32) c_ord[c] = c;   // valid even if ranks collide (NaN)
-    __syncwarp();
-    for (int c = lane; c < nc; c += 32) {   // rank by (value desc, index asc)
-      const double vc = c_val[c];
-      const int ic = c_idx[c];
-      int rank = 0;
-      for (int j = 0; j < nc; ++j) {
-        const double vj = c_val[j];
-        rank += (vj > vc || (vj == vc && c_idx[j] < ic)) ? 1 : 0;
-      }
-      if (rank < nc) c_ord[rank] = c;
-    }
-    __syncwarp();
-    // ---- tier 3: clusters closer than the fp64 bound, ordered exactly -----
-    const double margin64 = 2.000001 * r64;
-    int pos = 0;
-    const uint16_t* xbits = reinterpret_cast<const uint16_t*>(xrow);
-    while (got < k) {
-      int end = pos;
-      while (end + 1 < nc && !(c_val[c_ord[end]] - c_val[c_ord[end + 1]] > margin64)) ++end;
-      if (end == pos) {
-        put(c_idx[c_ord[pos]], c_val[c_ord[pos]]);
-        pos = end + 1;
-        continue;
-      }
-      const int need = min(end - pos + 1, k - got);
-      for (int q = 0; q < need; ++q) {
-        long long best[kLimbs];
-        int best_e = -1, best_slot = -1;
-        for (int m = pos; m <= end; ++m) {
-          const int e = c_idx[c_ord[m]];
-          if (e < 0) continue;   // already chosen
-          long long cur[kLimbs];
-          exact_logit(xbits, reinterpret_cast<const uint16_t*>(router_w) + static_cast<size_t>(e) * H,
-                      bias ? bias[e] : 0.f, H, cur);
-          int cmp = best_e < 0 ? 1 : exact_cmp(cur, best);
-          if (cmp > 0 || (cmp == 0 && e < best_e)) {
-#pragma unroll
-            for (int i = 0; i < kLimbs; ++i) best[i] = cur[i];
-            best_e = e;
-            best_slot = m;
-          }
+        for (int r = 0; r < 4; ++r) wrows[r] = router_w + static_cast<size_t>(c_idx[c + (r < nw ? r : 0)]) * H;
+        double dd[4];
+        if (mixed)
+          logits4<true>(xrow, wrows, nw, H, dd);
+        else
+          logits4<false>(xrow, wrows, nw, H, dd);
+        for (int r = 0; r < nw; ++r) {
+          const int e = c_idx[c + r];
+          const double b = bias ? static_cast<double>(bias[e]) : 0.0;
+          const double d = dd[r] + b;
+          rmx = fmax(rmx, (g * xn * wnorm_of(e) + 2.3e-16 * (fabs(d) + fabs(b))) * 1.001 + floor_err);
+          if (lane == 0) c_val[c + r] = d;
         }
-        put(best_e, c_val[c_ord[best_slot]]);
-        __syncwarp();
-        if (lane == 0) c_idx[c_ord[best_slot]] = -1;
-        __syncwarp();
       }
-      pos = end + 1;
+      __syncwarp();
+      rank_candidates(c_idx, c_ord, c_val, nc);
+      return rmx;
+    };
+    // tc_tier: first in mixed precision, which decides when every adjacent
+    // gap among the first k+1 exceeds twice its bound; otherwise (and for
+    // CUDA-core logits) in fp64
+    double margin = 2.000001 * evaluate(tc_tier);
+    if (tc_tier) {
+      bool bad = false;
+      for (int i = lane; i < k && i + 1 < nc; i += 32) bad |= !(c_val[c_ord[i]] - c_val[c_ord[i + 1]] > margin);
+      if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) atomicAdd(hdr + kHdrUncertain, 1u);
+        margin = 2.000001 * evaluate(false);
+      }
     }
+    // ---- tier 3: clusters closer than the margin, ordered exactly ----------
+    assemble_in_order(c_idx, c_ord, c_val, nc, k, margin, xrow, router_w, bias, H, got, put);
   }
 
   // renormalised weights of the selected experts: fp32 softmax values
-  // renormalised over the k; on the fp64 tier the same quantity from the
-  // fp64 logits, exp(d_j - max_j d) / sum_j (the full softmax's denominator
-  // cancels in the renormalisation)
+  // renormalised over the k; on tc_tier the same quantity from the
+  // re-evaluated logits, exp(d_j - max_j d) / sum_j (the full softmax's
+  // denominator cancels in the renormalisation)
   float p;
-  if (fp64_tier) {
+  if (tc_tier) {
     double dm = lane < k ? my_d : -1.0e300;
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) dm = fmax(dm, __shfl_xor_sync(0xffffffffu, dm, m));
@@ -779,7 +841,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
     const float* __restrict__ bias, const __nv_bfloat16* __restrict__ hidden,
     const __nv_bfloat16* __restrict__ router_w, int T, int H, int E, int k, float gamma, float ulast,
     int32_t* __restrict__ topk_ids, float* __restrict__ topk_w, unsigned char* __restrict__ cand,
-    uint32_t* __restrict__ hdr, AlignArgs aa, int with_align, int fp64_tier) {
+    uint32_t* __restrict__ hdr, AlignArgs aa, int with_align, int tc_tier) {
   extern __shared__ int align_hist[];
   __shared__ int s_last;
   pdl_wait();
@@ -787,7 +849,7 @@ __global__ void __launch_bounds__(256) router_topk_kernel(
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
   if (t < T)
     topk_token<kPer>(t, logits, xnorm, wnorm, amax_tok, rsplit, nsplit, bias, hidden, router_w, T, H,
-                     E, k, gamma, ulast, topk_ids, topk_w, cand, hdr, fp64_tier != 0);
+                     E, k, gamma, ulast, topk_ids, topk_w, cand, hdr, tc_tier != 0);
   if (!with_align) return;
   __syncthreads();   // every top-k of this CTA is stored
   if (threadIdx.x == 0) {
@@ -814,7 +876,7 @@ static cudaError_t launch_logits(const RouterArgs& a, cudaStream_t st) {
 
 template <int kPer>
 static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, int nsplit,
-                               cudaStream_t st, const AlignArgs* aa = nullptr, bool fp64_tier = false) {
+                               cudaStream_t st, const AlignArgs* aa = nullptr, bool tc_tier = false) {
   const int smem = aa ? 8 * a.E * 4 : 0;   // the align's per-warp histograms (8 warps)
   auto kern = router_topk_kernel<kPer>;
   if (smem > 0) {
@@ -823,7 +885,7 @@ static cudaError_t launch_topk(const RouterArgs& a, float gamma, float ulast, in
   }
   return launch_pdl(kern, dim3((a.T + 7) / 8), dim3(256), smem, st, a.logits, a.xnorm, a.wnorm, a.amax_tok,
                     a.rsplit, nsplit, a.bias, a.hidden, a.router_w, a.T, a.H, a.E, a.k, gamma, ulast,
-                    a.topk_ids, a.topk_w, a.cand, a.hdr, aa ? *aa : AlignArgs{}, aa ? 1 : 0, fp64_tier ? 1 : 0);
+                    a.topk_ids, a.topk_w, a.cand, a.hdr, aa ? *aa : AlignArgs{}, aa ? 1 : 0, tc_tier ? 1 : 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -908,12 +970,20 @@ static cudaError_t launch_logits_tiled(const RouterArgs& a, int nsplit, cudaStre
                     a.logits, a.xnorm, a.wnorm, a.amax_tok, a.rsplit);
 }
 
-cudaError_t launch_router_topk(const RouterArgs& a, float gamma, float ulast, cudaStream_t st) {
-  // logits from the tensor cores: every token ranked and weighted on the fp64 tier
-  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, 1, st, nullptr, true);
-  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, 1, st, nullptr, true);
-  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, 1, st, nullptr, true);
-  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, 1, st, nullptr, true);
+cudaError_t launch_router_topk_tc(const RouterArgs& a, float gamma, float ulast, cudaStream_t st,
+                                  const AlignArgs* fuse_align, bool* fused) {
+  if (fused) *fused = false;
+  const AlignArgs* aa = nullptr;
+  if (fuse_align != nullptr && fused != nullptr && a.E <= 256 &&
+      static_cast<long long>(a.T) * a.k < kAlignSliceMin) {
+    aa = fuse_align;
+    *fused = true;
+  }
+  // logits from the tensor cores: every token's candidates re-evaluated
+  if (a.E <= 64) return launch_topk<2>(a, gamma, ulast, 1, st, aa, true);
+  if (a.E <= 128) return launch_topk<4>(a, gamma, ulast, 1, st, aa, true);
+  if (a.E <= 256) return launch_topk<8>(a, gamma, ulast, 1, st, aa, true);
+  return launch_topk<kMaxExperts / 32>(a, gamma, ulast, 1, st, aa, true);
 }
 
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align, bool* fused) {

@@ -402,3 +402,19 @@ def test_fused_ffn_matches_two_launch_path(cuda_ok, name):
     assert_output_close(two, ref, fp8=False)
     d = (fused.float() - two.float()).abs().max().item()
     assert d <= 2e-2 * max(ref["out"].std(), 1e-6), d
+
+
+def test_route_tests_on_tensor_core_tier(cuda_ok):
+    """The routing tests above again, every call's logits from the tensor
+    cores (MOE_ROUTER=tc; the path is fixed per process, so in a child
+    process): near ties, duplicate rows, equal logits and the bias alone then
+    go through the fp64 candidate tier and the exact tier from the loose
+    tensor-core bound."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_ROUTER="tc")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-m", "gpu", "-x", "-q", "-k",
+                        "route and not tensor_core_tier", "-p", "no:cacheprovider"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
