@@ -80,14 +80,16 @@ def peaks():
 
 
 def kernel_traffic(workload):
-    """ncu DRAM bytes per launch of the w13 kernel, if captured for this source."""
+    """ncu DRAM bytes per launch of the workload's roofline kernel, if captured
+    for the current source of that kernel (the entry names its file)."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(workload)
     if not d:
         return None
-    if code_sha(os.path.join(ROOT, "mixture_experts_layer_counts_b200", "csrc", "gemm.cu")) != d.get("gemm_cu_sha"):
+    src = os.path.join(ROOT, "mixture_experts_layer_counts_b200", "csrc", d.get("code_file", "gemm.cu"))
+    if not os.path.exists(src) or code_sha(src) != d.get("code_sha"):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -718,6 +720,8 @@ def main():
     ap.add_argument("--workload", default=HEADLINE, choices=list(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--only-headline", action="store_true", help="skip the other workloads")
+    ap.add_argument("--rope-only", action="store_true",
+                    help="time the fused inverse-RoPE + FP8 kernel alone (one JSON line)")
     ap.add_argument("--route-only", action="store_true",
                     help="time the router alone on the workload's hidden states (no expert weights)")
     ap.add_argument("--sweep-orientation", action="store_true",
@@ -753,6 +757,9 @@ def main():
         return
     if args.route_only:
         route_only(wl, local, args.steps)
+        return
+    if args.rope_only:
+        print(json.dumps({"inv_rope_fp8": measure_inv_rope(local, args.steps)}), flush=True)
         return
     try:
         run_ours(args, wl, rank, world, local)

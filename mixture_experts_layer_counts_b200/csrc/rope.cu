@@ -29,7 +29,8 @@
 // which also gives a zero quotient the sign of y (the plain order turns -0
 // into +0); the codes of the negated quotients are flipped back with one XOR
 // per four codes (E4M3 is sign-magnitude and its rounding symmetric).  The
-// two lanes of each step share one packed fp32x2 instruction (sm_100).  The
+// two lanes of each step share one packed fp32x2 instruction (sm_100), the
+// pair kept in one 64-bit register through the three steps.  The
 // rotation stays in scalar multiplies and adds with explicit rounding, so no
 // product is fused into the sum.
 //
@@ -60,20 +61,26 @@ __device__ __forceinline__ uint32_t e4m3x4(float a, float b, float c, float d) {
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-// Packed fp32x2 multiply and fused multiply-add, round-to-nearest-even (lane x in the low half).
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
-  float2 d;
-  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+// Packed fp32x2 arithmetic on 64-bit registers (lane x in the low half).
+__device__ __forceinline__ unsigned long long pack2(float x, float y) {
+  unsigned long long d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "f"(x), "f"(y));
   return d;
 }
-
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+__device__ __forceinline__ float2 unpack2(unsigned long long v) {
   float2 d;
-  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "mov.b64 rc, {%6, %7};\n\tfma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
-      : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(d.x), "=f"(d.y) : "l"(v));
+  return d;
+}
+__device__ __forceinline__ unsigned long long mul2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long fma2(unsigned long long a, unsigned long long b,
+                                                   unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
 
@@ -135,13 +142,13 @@ __global__ void __launch_bounds__(256, 6) inv_rope_fp8_kernel(
       float d0[8], d1[8];
       if (scale >= 0x1p-100f && scale <= 0x1p100f) {
         const float nr = -__frcp_rn(scale);
-        const float2 NR = make_float2(nr, nr), SC = make_float2(scale, scale);
+        const unsigned long long NR = pack2(nr, nr), SC = pack2(scale, scale);
 #pragma unroll
         for (int i = 0; i < 8; i += 2) {
-          const float2 Y0 = make_float2(y0[i], y0[i + 1]), Y1 = make_float2(y1[i], y1[i + 1]);
-          const float2 n0 = mul2(Y0, NR), n1 = mul2(Y1, NR);
-          const float2 e0 = fma2(n0, SC, Y0), e1 = fma2(n1, SC, Y1);
-          const float2 q0 = fma2(e0, NR, n0), q1 = fma2(e1, NR, n1);
+          const unsigned long long Y0 = pack2(y0[i], y0[i + 1]), Y1 = pack2(y1[i], y1[i + 1]);
+          const unsigned long long n0 = mul2(Y0, NR), n1 = mul2(Y1, NR);
+          const unsigned long long e0 = fma2(n0, SC, Y0), e1 = fma2(n1, SC, Y1);
+          const float2 q0 = unpack2(fma2(e0, NR, n0)), q1 = unpack2(fma2(e1, NR, n1));
           d0[i] = q0.x; d0[i + 1] = q0.y; d1[i] = q1.x; d1[i + 1] = q1.y;
         }
         qa = make_uint2(e4m3x4(d0[0], d0[1], d0[2], d0[3]) ^ 0x80808080u,
