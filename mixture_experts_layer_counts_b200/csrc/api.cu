@@ -385,7 +385,11 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
       g.amax_cta = amax_cta + (any_swap ? grid : 0);
       g.flags = flags + 1 * kMaxSlots;
       requant_args(g, true);
-      MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
+      if (w13_pair2sm_supported(I, fp8)) {
+        MOE_TRY(cuda_status(launch_w13_pair2sm(tw13n, txn, g, grid, st)));
+      } else {
+        MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW13, fp8, tw13n, txn, g, grid, st)));
+      }
     }
     record(dbg, 4, st);   // (the FP8 requantisation ran at the end of the gate/up GEMM)
     record(dbg, 5, st);
