@@ -256,7 +256,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   const bool any_normal = T > tau;
 
   // tensor maps (weights and grouped activations), built before any launch
-  CUtensorMap tw13s, tw13n, tw2s, tw2n, txs, txn, tis, tin;
+  CUtensorMap tw13s, tw13n, tw2s, tw2n, tw2p, txs, txn, tis, tin;
   const long long w13_rows = static_cast<long long>(E) * 2 * I;
   const long long w2_rows = static_cast<long long>(E) * H;
   void* xperm = at<void>(ws, L.xperm);
@@ -270,6 +270,7 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
   if (any_normal) {
     MOE_TRY(make_tmap(&tw13n, w13, fp8, H, w13_rows, gemm_weight_box_rows(Orient::kNormal, Proj::kW13)));
     MOE_TRY(make_tmap(&tw2n, w2, fp8, I, w2_rows, gemm_weight_box_rows(Orient::kNormal, Proj::kW2)));
+    if (w2_pair2sm_supported(H, fp8)) MOE_TRY(make_tmap(&tw2p, w2, fp8, I, w2_rows, 128));
     MOE_TRY(make_tmap(&txn, xperm, fp8, H, A, gemm_token_box_rows(Orient::kNormal)));
     MOE_TRY(make_tmap(&tin, inter, fp8, I, A, gemm_token_box_rows(Orient::kNormal)));
   }
@@ -403,11 +404,17 @@ moe_status_t forward_impl(const void* hidden, const void* router_w, const float*
     }
     if (any_normal) {
       GemmArgs g = g2;
-      g.chunks = at<int4>(ws, gemm_w2_pair() ? L.chunks_pair : L.chunks_normal);
-      g.nchunks = hdr + (gemm_w2_pair() ? kHdrChunksPair : kHdrChunksNormal);
-      g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
       g.flags = flags + 3 * kMaxSlots;
-      MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
+      if (w2_pair2sm_supported(H, fp8)) {
+        g.chunks = at<int4>(ws, L.chunks_pair);
+        g.nchunks = hdr + kHdrChunksPair;
+        MOE_TRY(cuda_status(launch_w2_pair2sm(tw2p, tin, g, grid, st)));
+      } else {
+        g.chunks = at<int4>(ws, gemm_w2_pair() ? L.chunks_pair : L.chunks_normal);
+        g.nchunks = hdr + (gemm_w2_pair() ? kHdrChunksPair : kHdrChunksNormal);
+        g.mtiles = H / gemm_weight_box_rows(Orient::kNormal, Proj::kW2);
+        MOE_TRY(cuda_status(launch_gemm(Orient::kNormal, Proj::kW2, fp8, tw2n, tin, g, grid, st)));
+      }
     }
   }
   record(dbg, 6, st);

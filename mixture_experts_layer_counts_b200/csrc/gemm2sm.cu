@@ -1,27 +1,31 @@
-// Gate/up GEMM of prefill-sized batches (normal orientation, bf16) on CTA
+// Expert GEMMs of prefill-sized batches (normal orientation, bf16) on CTA
 // pairs: one tcgen05 MMA spans the tensor cores of two SMs (cta_group::2).
 //
 // Why.  The single-CTA normal-orientation kernel (gemm.cu) holds a 256-token
 // x 256-weight-row accumulator in one SM's TMEM (all 512 columns) and stages
-// 64 KB of operands per 64-element K atom (two token tiles, the gate and up
-// tiles).  Its ring of three such stages cannot cover the latency of weight
-// lines that miss L2, so the tensor pipe idles about a third of the time.  A
-// pair of CTAs computes a 256-token x 512-weight-row tile (gate 256 + up 256)
-// with M = 256 MMAs whose A operand (tokens) is split by rows between the two
-// SMs and whose B operand (weight rows) is split by rows too: each CTA stages
-// 128 token rows, 128 gate rows and 128 up rows, 48 KB per K atom for the
-// same MMA work per SM, so four stages fit and 25 % fewer bytes cross from L2
-// per multiply-add.
+// 64 KB of operands per 64-element K atom (two token tiles, 256 weight rows).
+// Its ring of three such stages cannot cover the latency of weight lines that
+// miss L2, so the tensor pipe idles about a third of the time.  A pair of CTAs
+// computes a 256-token x 512-weight-row tile with M = 256, N = 256 MMAs whose
+// A operand (tokens) is split by rows between the two SMs and whose B operand
+// (weight rows) is split by rows too: each CTA stages 128 token rows and two
+// 128-row weight tiles, 48 KB per K atom for the same MMA work per SM, so
+// four stages fit and 25 % fewer bytes cross from L2 per multiply-add.
+//   Gate/up (kW2 = false): the two weight tiles are rows [128 r, +128) of the
+//   gate and of the up part of a 256-row slice of I; accumulator columns
+//   [0, 256) gate, [256, 512) up; the epilogue writes h = SiLU(g) u (bf16).
+//   Down (kW2 = true): rows [128 r, +128) of each 256-row half of a 512-row
+//   slice of H; the epilogue writes the router-weighted fp32 rows to the
+//   assignment's slot row of ysc, as the one-CTA down GEMM does.
 //
-// Unit = (expert, 256-row slice of I, 256-token chunk), dealt round-robin
-// over the pairs in the grouped order of unit_coords (expert, then weight
-// slice, then chunk), so the chunks sharing a weight slice run together.
-// CTA rank r of the pair owns token rows [128 r, 128 r + 128) of the chunk
-// and weight rows [128 r, 128 r + 128) of the gate and the up slice.
+// Unit = (expert, weight slice, 256-token chunk), dealt round-robin over the
+// pairs in the grouped order of unit_coords (expert, then weight slice, then
+// chunk), so the chunks sharing a weight slice run together.  CTA rank r of
+// the pair owns token rows [128 r, 128 r + 128) of the chunk.
 //
 // Roles in each CTA: warp 0 lane 0 TMA producer, warp 1 TMEM allocation (both
 // CTAs) and MMA issue (rank 0 only), warps 2..9 epilogue (two per TMEM lane
-// quadrant, each half of the 256 columns of h).
+// quadrant, each half of the accumulator columns).
 // Barriers (same shared-memory offsets in both CTAs):
 //   full[s]   rank 0's: one arrival (rank 0's producer, expecting the bytes of
 //             both CTAs' copies, which all complete on rank 0's barrier);
@@ -29,13 +33,6 @@
 //             CTA's barrier);
 //   acc_full  each CTA's own: rank 0 commits after the unit's last K atom;
 //   acc_empty rank 0's: one arrival per epilogue warp of both CTAs.
-// The producers' arrivals stay inside the CTA: rank 0 alone arms full[s] with
-// the bytes of both CTAs' copies (a cluster-scope release on every stage, as
-// in a two-arrival form, cost about a microsecond per stage and left the
-// ring serialised).
-// Every wait is bounded (wait_cluster, mbar_wait); a CTA that gives up raises its abort
-// flag, drains what it has in flight, and both CTAs meet at the final cluster
-// barrier before TMEM is released.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -146,9 +143,10 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
 
 }  // namespace
 
+template <bool kW2>
 __global__ void __launch_bounds__(kP2Threads, 1)
-    w13_pair2sm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
-                       const GemmArgs a) {
+    gemm_pair2sm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                        const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
@@ -217,7 +215,12 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       int mt;
       unit_coords<true, kPairTokens>(a, u, ch, mt);
       const int e = ch.x, p0 = ch.y;
-      const int grow = e * a.w_rows_per_expert + mt * 2 * kP2Rows + static_cast<int>(rank) * kP2Rows;
+      // gate/up: rows [128 r, +128) of the gate and of the up slice (second
+      // tile up_offset further); down: rows [128 r, +128) of each 256-row
+      // half of the 512-row slice of H (second tile 256 further)
+      const int slice = kW2 ? 4 * kP2Rows : 2 * kP2Rows;
+      const int grow = e * a.w_rows_per_expert + mt * slice + static_cast<int>(rank) * kP2Rows;
+      const int second = kW2 ? 2 * kP2Rows : a.up_offset;
       const int trow = p0 + static_cast<int>(rank) * kP2Tok;
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, a.hdr, kSiteProducerEmpty, a.timeout_ns)) {
@@ -232,7 +235,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         const int kc = kb * 64;
         tma_load_2d_pair(st, &tm_x, fb, kc, trow, pol_x);
         tma_load_2d_pair(st + kP2Tile, &tm_w, fb, kc, grow, pol_w);
-        tma_load_2d_pair(st + 2 * kP2Tile, &tm_w, fb, kc, grow + a.up_offset, pol_w);
+        tma_load_2d_pair(st + 2 * kP2Tile, &tm_w, fb, kc, grow + second, pol_w);
         if (++stage == kP2Stages) {
           stage = 0;
           phase ^= 1u;
@@ -295,8 +298,11 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------------------ epilogue --
-    // h[token, i] = SiLU(g) * u for this CTA's 128 token rows; warp half hx
-    // takes columns [128 hx, 128 hx + 128) of the 256-row slice of I.
+    // this CTA's 128 token rows; warp half hx takes half of the accumulator
+    // columns.  Gate/up: h[token, i] = SiLU(g) * u over the 256-row slice of I
+    // (gate at columns [0, 256), up at [256, 512)), bf16 rows of `inter`.
+    // Down: the 512 columns of the H slice times the router weight, fp32 rows
+    // to the assignment's slot row f of ysc (streaming stores).
     const int q = warp & 3;
     const int hx = (warp - 2) >> 2;
     float* sw = epi + (warp - 2) * 32 * kP2EpiLd;
@@ -314,34 +320,61 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       const int p0 = ch.y, nv = ch.z;
       const int rb = static_cast<int>(rank) * kP2Tok + q * 32;   // first chunk row of this warp's block
       const uint32_t th = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-      const int i0 = mt * 2 * kP2Rows;
-      for (int c0 = hx * kP2Rows; c0 < (rb < nv ? (hx + 1) * kP2Rows : 0); c0 += 16) {
-        float v[2][16];
-        tmem_ld16x2_wait(th + c0, th + 2 * kP2Rows + c0, v[0], v[1]);
-        float h[16];
+      if constexpr (!kW2) {
+        const int i0 = mt * 2 * kP2Rows;
+        for (int c0 = hx * kP2Rows; c0 < (rb < nv ? (hx + 1) * kP2Rows : 0); c0 += 16) {
+          float v[2][16];
+          tmem_ld16x2_wait(th + c0, th + 2 * kP2Rows + c0, v[0], v[1]);
+          float h[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) h[j] = __fdividef(v[0][j], 1.0f + __expf(-v[0][j])) * v[1][j];
+          for (int j = 0; j < 16; ++j) h[j] = __fdividef(v[0][j], 1.0f + __expf(-v[0][j])) * v[1][j];
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          uint32_t w4[4];
+          for (int j = 0; j < 2; ++j) {
+            uint32_t w4[4];
 #pragma unroll
-          for (int m = 0; m < 4; ++m) {
-            __nv_bfloat162 b2 = __floats2bfloat162_rn(h[8 * j + 2 * m], h[8 * j + 2 * m + 1]);
-            w4[m] = *reinterpret_cast<uint32_t*>(&b2);
+            for (int m = 0; m < 4; ++m) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(h[8 * j + 2 * m], h[8 * j + 2 * m + 1]);
+              w4[m] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(su + lane * kP2EpiLd + 4 * j) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-          *reinterpret_cast<uint4*>(su + lane * kP2EpiLd + 4 * j) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-        __syncwarp();
-        // 2 lanes per row (32 B), 16 rows per instruction
+          __syncwarp();
+          // 2 lanes per row (32 B), 16 rows per instruction
 #pragma unroll
-        for (int r0 = 0; r0 < 32; r0 += 16) {
-          const int r = r0 + (lane >> 1);
-          const uint4 val = *reinterpret_cast<const uint4*>(su + r * kP2EpiLd + 4 * (lane & 1));
-          if (rb + r < nv)
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + static_cast<size_t>(p0 + rb + r) * a.ld_out +
-                                      i0 + c0 + 8 * (lane & 1)) = val;
+          for (int r0 = 0; r0 < 32; r0 += 16) {
+            const int r = r0 + (lane >> 1);
+            const uint4 val = *reinterpret_cast<const uint4*>(su + r * kP2EpiLd + 4 * (lane & 1));
+            if (rb + r < nv)
+              *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) +
+                                        static_cast<size_t>(p0 + rb + r) * a.ld_out + i0 + c0 + 8 * (lane & 1)) = val;
+          }
+          __syncwarp();
         }
-        __syncwarp();
+      } else {
+        const int f = rb + lane < nv ? a.perm[p0 + rb + lane] : -1;
+        const bool valid = f >= 0 && f < a.num_assign;
+        const float wt = valid ? a.topk_w[f] : 0.f;
+        const int h0 = mt * 4 * kP2Rows;
+        for (int c0 = hx * 2 * kP2Rows; c0 < (rb < nv ? (hx + 1) * 2 * kP2Rows : 0); c0 += 16) {
+          float v[16];
+          tmem_ld16_wait(th + c0, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<float4*>(sw + lane * kP2EpiLd + 4 * j) =
+                make_float4(v[4 * j] * wt, v[4 * j + 1] * wt, v[4 * j + 2] * wt, v[4 * j + 3] * wt);
+          __syncwarp();
+          // 4 lanes per row (64 B), 8 rows per instruction
+#pragma unroll
+          for (int r0 = 0; r0 < 32; r0 += 8) {
+            const int r = r0 + (lane >> 2);
+            const int fr = __shfl_sync(0xffffffffu, f, r);
+            const float4 val = *reinterpret_cast<const float4*>(sw + r * kP2EpiLd + 4 * (lane & 3));
+            if (fr >= 0 && fr < a.num_assign)
+              __stcs(reinterpret_cast<float4*>(static_cast<float*>(a.out) + static_cast<size_t>(fr) * a.ld_out +
+                                               h0 + c0 + 4 * (lane & 3)), val);
+          }
+          __syncwarp();
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -356,18 +389,25 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   if (warp == 1) tmem_dealloc_pair(tmem_base, 512);
 }
 
+static int env_on(const char* name) {
+  const char* s = std::getenv(name);
+  return (s && std::atoi(s) == 0) ? 0 : 1;
+}
+
 bool w13_pair2sm_supported(int I, bool fp8) {
-  static int v = -1;
-  if (v < 0) {
-    const char* s = std::getenv("MOE_W13_2SM");
-    v = (s && std::atoi(s) == 0) ? 0 : 1;
-  }
+  static const int v = env_on("MOE_W13_2SM");
   return v == 1 && !fp8 && I % (2 * kP2Rows) == 0;
 }
 
-cudaError_t launch_w13_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
-                               cudaStream_t st) {
-  auto kern = w13_pair2sm_kernel;
+bool w2_pair2sm_supported(int H, bool fp8) {
+  static const int v = env_on("MOE_W2_2SM");
+  return v == 1 && !fp8 && H % (4 * kP2Rows) == 0;
+}
+
+template <bool kW2>
+static cudaError_t launch_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
+                                  cudaStream_t st) {
+  auto kern = gemm_pair2sm_kernel<kW2>;
   cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), kP2Smem);
   if (err != cudaSuccess) return err;
   // as many CTA pairs as can be resident at once (one CTA per SM)
@@ -409,8 +449,19 @@ cudaError_t launch_w13_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, con
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   GemmArgs g = a;
-  g.mtiles = a.up_offset / (2 * kP2Rows);   // slices of I per CTA pair
+  // slices per CTA pair: 256 rows of I (gate/up) or 512 rows of H (down)
+  g.mtiles = kW2 ? a.w_rows_per_expert / (4 * kP2Rows) : a.up_offset / (2 * kP2Rows);
   return cudaLaunchKernelEx(&cfg, kern, tw, tx, g);
+}
+
+cudaError_t launch_w13_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
+                               cudaStream_t st) {
+  return launch_pair2sm<false>(tw, tx, a, max_ctas, st);
+}
+
+cudaError_t launch_w2_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
+                              cudaStream_t st) {
+  return launch_pair2sm<true>(tw, tx, a, max_ctas, st);
 }
 
 }  // namespace moe

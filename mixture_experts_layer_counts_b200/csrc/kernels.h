@@ -175,11 +175,16 @@ enum class Proj { kW13, kW2 };
 cudaError_t launch_gemm(Orient o, Proj p, bool fp8, const CUtensorMap& tm_w,
                         const CUtensorMap& tm_x, const GemmArgs& a, int grid, cudaStream_t st);
 bool gemm_w2_pair();
-// Gate/up GEMM of the normal orientation on CTA pairs (gemm2sm.cu): bf16, I a
-// multiple of 256; MOE_W13_2SM=0 keeps the one-CTA kernel (for measurements).
+// Normal-orientation GEMMs on CTA pairs (gemm2sm.cu), bf16, 256-token chunks:
+// gate/up with I a multiple of 256, down with H a multiple of 512.  Both take
+// 128-row boxes in their tensor maps.  MOE_W13_2SM=0 / MOE_W2_2SM=0 keep the
+// one-CTA kernels (for measurements).
 bool w13_pair2sm_supported(int I, bool fp8);
+bool w2_pair2sm_supported(int H, bool fp8);
 cudaError_t launch_w13_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
-                               cudaStream_t st);                 // normal down GEMM on 256-token chunks (two M tiles)
+                               cudaStream_t st);
+cudaError_t launch_w2_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
+                              cudaStream_t st);                 // normal down GEMM on 256-token chunks (two M tiles)
 int gemm_token_box_rows(Orient o);   // rows per TMA box of the token operand
 int gemm_swap_chunk();               // largest token chunk of the swap-AB kernels
 int gemm_weight_box_rows(Orient o, Proj p);
