@@ -497,7 +497,9 @@ def measure_workload(name, wl, args, rank, world, local, steps_exact=None):
     if tensor_bound:
         mult = 2.0 if dt == 1 else 1.0      # E4M3: the nominal fp8 / bf16 ratio
         ach = w13_flops / w13_s / 1e12
-        roof = {"kernel": "grouped_gemm_kernel<normal, w13>", "bound": "tensor", "achieved": ach,
+        pair = dt == 0 and I % 256 == 0 and os.environ.get("MOE_W13_2SM", "1") != "0"
+        roof = {"kernel": "gemm_pair2sm_kernel<W13> (CTA pairs)" if pair else "grouped_gemm_kernel<normal, w13>",
+                "bound": "tensor", "achieved": ach,
                 "peak": mult * pk["bf16"], "unit": "TFLOP/s", "frac": ach / (mult * pk["bf16"]),
                 "peak_kind": pk["kind"] + (" bf16 burst" if mult == 1 else " bf16 burst x 2 (fp8 nominal ratio)"),
                 "peak_sustained": mult * pk["bf16_sustained"],
