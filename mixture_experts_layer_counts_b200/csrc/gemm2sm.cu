@@ -14,9 +14,15 @@
 //   Gate/up (kW2 = false): the two weight tiles are rows [128 r, +128) of the
 //   gate and of the up part of a 256-row slice of I; accumulator columns
 //   [0, 256) gate, [256, 512) up; the epilogue writes h = SiLU(g) u (bf16).
-//   Down (kW2 = true): rows [128 r, +128) of each 256-row half of a 512-row
-//   slice of H; the epilogue writes the router-weighted fp32 rows to the
-//   assignment's slot row of ysc, as the one-CTA down GEMM does.
+//   Down (kW2 = true): the epilogue writes the router-weighted fp32 rows to
+//   the assignment's slot row of ysc, as the one-CTA down GEMM does.  Its K
+//   loop is short (I / 64 atoms) and its epilogue heavy, so by default
+//   (kDB) a pair tile is 256 tokens x 256 rows of H, one weight tile of
+//   rows [128 r, +128) per CTA and stage (six 32 KB stages), in two
+//   256-column accumulators: a unit's epilogue overlaps the next unit's
+//   MMAs (measured 570-594 us against 603-613 us for the 512-row form at
+//   prefill-zipf; MOE_W2_2SM_DB=0 selects that form: rows [128 r, +128) of
+//   each 256-row half of a 512-row slice, one 512-column accumulator).
 //
 // Unit = (expert, weight slice, 256-token chunk), dealt round-robin over the
 // pairs in the grouped order of unit_coords (expert, then weight slice, then
@@ -50,14 +56,27 @@ namespace {
 constexpr int kP2Tok = 128;                   // token rows per CTA
 constexpr int kP2Rows = 128;                  // gate (and up) weight rows per CTA
 constexpr int kP2Tile = 128 * kAtomBytes;     // 16 KB: one 128-row operand tile of a K atom
-constexpr int kP2Stage = 3 * kP2Tile;         // A, B gate, B up
-constexpr int kP2Stages = 4;
 constexpr int kP2EpiWarps = 8;
 constexpr int kP2Threads = 64 + 32 * kP2EpiWarps;
 constexpr int kP2EpiLd = 20;                  // staged 32 x 16 block, rows padded to 20 words
 constexpr int kP2EpiBytes = kP2EpiWarps * 32 * kP2EpiLd * 4;
-constexpr int kP2Smem = kP2Stages * kP2Stage + 1024 /*align*/ + 256 /*barriers*/ + kP2EpiBytes;
-static_assert(kP2Smem <= 232448, "shared memory");
+
+// Per form: kB weight tiles per stage (two: gate and up, or two halves of
+// H; one: the down GEMM's 256-row slice of H), the ring depth, and the
+// accumulator buffers (one of 512 columns, or two of 256 so the epilogue of
+// a unit overlaps the next unit's MMAs).
+template <bool kW2, bool kDB>
+struct P2 {
+  static constexpr int kB = kDB ? 1 : 2;
+  static constexpr int kStage = (1 + kB) * kP2Tile;
+  static constexpr int kStages = kDB ? 6 : 4;
+  static constexpr int kBufs = kDB ? 2 : 1;
+  static constexpr int kAccCols = kB * 2 * kP2Rows;               // per buffer
+  static constexpr int kSlice = kW2 ? kB * 2 * kP2Rows : 2 * kP2Rows;   // weight rows of a unit's slice
+  static constexpr int kSmem = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/ + kP2EpiBytes;
+  static_assert(kSmem <= 232448, "shared memory");
+  static_assert(!kDB || kW2, "the double-buffered form is the down GEMM's");
+};
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -143,34 +162,37 @@ __device__ __forceinline__ void commit_pair(uint32_t bar) {
 
 }  // namespace
 
-template <bool kW2>
+template <bool kW2, bool kDB>
 __global__ void __launch_bounds__(kP2Threads, 1)
     gemm_pair2sm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                         const GemmArgs a) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
+  using C = P2<kW2, kDB>;
   uint8_t* tiles = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + kP2Stages * kP2Stage);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(tiles + C::kStages * C::kStage);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kP2Stages;
-  uint64_t* acc_full = bars + 2 * kP2Stages;
-  uint64_t* acc_empty = acc_full + 1;
-  uint64_t* drain = acc_empty + 1;
+  uint64_t* empty = bars + C::kStages;
+  uint64_t* acc_full = bars + 2 * C::kStages;
+  uint64_t* acc_empty = acc_full + C::kBufs;
+  uint64_t* drain = acc_empty + C::kBufs;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* epi = reinterpret_cast<float*>(tiles + kP2Stages * kP2Stage + 256);
+  float* epi = reinterpret_cast<float*>(tiles + C::kStages * C::kStage + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
   const bool lead = rank == 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kP2Stages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 2 * kP2EpiWarps);
+    for (int b = 0; b < C::kBufs; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kP2EpiWarps);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -199,7 +221,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 
   // rank 0's barriers as shared::cluster addresses (rank 0 itself included)
   auto full0 = [&](int s) { return peer_addr(&full[s], 0); };
-  const uint32_t acc_empty0 = peer_addr(acc_empty, 0);
+  uint32_t acc_empty0[C::kBufs];
+  for (int b = 0; b < C::kBufs; ++b) acc_empty0[b] = peer_addr(&acc_empty[b], 0);
 
   if (warp == 0 && lane == 0) {
     // ------------------------------------------------------- TMA producer --
@@ -218,8 +241,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       // gate/up: rows [128 r, +128) of the gate and of the up slice (second
       // tile up_offset further); down: rows [128 r, +128) of each 256-row
       // half of the 512-row slice of H (second tile 256 further)
-      const int slice = kW2 ? 4 * kP2Rows : 2 * kP2Rows;
-      const int grow = e * a.w_rows_per_expert + mt * slice + static_cast<int>(rank) * kP2Rows;
+      const int grow = e * a.w_rows_per_expert + mt * C::kSlice + static_cast<int>(rank) * kP2Rows;
       const int second = kW2 ? 2 * kP2Rows : a.up_offset;
       const int trow = p0 + static_cast<int>(rank) * kP2Tok;
       for (int kb = kb0; kb < kb1; ++kb) {
@@ -230,13 +252,13 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         const uint32_t fb = full0(stage);
         // rank 0 expects both CTAs' bytes; rank 1's copies may land first
         // (the transaction count goes below zero until rank 0 arrives)
-        if (lead) mbar_arrive_expect_tx(&full[stage], 2 * kP2Stage);
-        uint8_t* st = tiles + stage * kP2Stage;
+        if (lead) mbar_arrive_expect_tx(&full[stage], 2 * C::kStage);
+        uint8_t* st = tiles + stage * C::kStage;
         const int kc = kb * 64;
         tma_load_2d_pair(st, &tm_x, fb, kc, trow, pol_x);
         tma_load_2d_pair(st + kP2Tile, &tm_w, fb, kc, grow, pol_w);
-        tma_load_2d_pair(st + 2 * kP2Tile, &tm_w, fb, kc, grow + second, pol_w);
-        if (++stage == kP2Stages) {
+        if constexpr (C::kB == 2) tma_load_2d_pair(st + 2 * kP2Tile, &tm_w, fb, kc, grow + second, pol_w);
+        if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
@@ -245,12 +267,16 @@ __global__ void __launch_bounds__(kP2Threads, 1)
   } else if (warp == 1 && lane == 0 && lead) {
     // ------------------------------------------------ MMA issuer (rank 0) --
     const uint32_t idesc = idesc_f32acc(1u, 2 * kP2Tok, 2 * kP2Rows);   // M = 256, N = 256, bf16
-    uint32_t empty_bar[kP2Stages][2];
-    for (int s = 0; s < kP2Stages; ++s) {
+    uint32_t empty_bar[C::kStages][2];
+    for (int s = 0; s < C::kStages; ++s) {
       empty_bar[s][0] = peer_addr(&empty[s], 0);
       empty_bar[s][1] = peer_addr(&empty[s], 1);
     }
-    const uint32_t accf0 = peer_addr(acc_full, 0), accf1 = peer_addr(acc_full, 1);
+    uint32_t accf[C::kBufs][2];
+    for (int b = 0; b < C::kBufs; ++b) {
+      accf[b][0] = peer_addr(&acc_full[b], 0);
+      accf[b][1] = peer_addr(&acc_full[b], 1);
+    }
     int stage = 0;
     uint32_t phase = 0;
     int it = 0;
@@ -258,11 +284,14 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     Segments seg = seg0;
     int u, kb0, kb1;
     while (ok && seg.next(u, kb0, kb1)) {
-      if (!wait_cluster(acc_empty, (it & 1) ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty, a.timeout_ns)) {
+      const int buf = it % C::kBufs;
+      if (!wait_cluster(&acc_empty[buf], ((it / C::kBufs) & 1) ^ 1u, abort_flag, a.hdr, kSiteMmaAccEmpty,
+                        a.timeout_ns)) {
         ok = false;
         break;
       }
       ++it;
+      const uint32_t d0 = tmem_base + buf * C::kAccCols;
       tc_fence_after();
       for (int kb = kb0; kb < kb1; ++kb) {
         if (!mbar_wait(&full[stage], phase, abort_flag, a.hdr, kSiteMmaFull, a.timeout_ns)) {
@@ -270,25 +299,26 @@ __global__ void __launch_bounds__(kP2Threads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t st = smem_u32(tiles + stage * kP2Stage);
+        const uint32_t st = smem_u32(tiles + stage * C::kStage);
 #pragma unroll
         for (int kk = 0; kk < kAtomBytes / 32; ++kk) {
           const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
           const uint32_t off = kk * 32;
-          mma_pair(tmem_base, sdesc_sw128(st + off), sdesc_sw128(st + kP2Tile + off), idesc, acc);
-          mma_pair(tmem_base + 2 * kP2Rows, sdesc_sw128(st + off), sdesc_sw128(st + 2 * kP2Tile + off), idesc, acc);
+          mma_pair(d0, sdesc_sw128(st + off), sdesc_sw128(st + kP2Tile + off), idesc, acc);
+          if constexpr (C::kB == 2)
+            mma_pair(d0 + 2 * kP2Rows, sdesc_sw128(st + off), sdesc_sw128(st + 2 * kP2Tile + off), idesc, acc);
         }
         issued = true;
         commit_pair(empty_bar[stage][0]);
         commit_pair(empty_bar[stage][1]);
-        if (++stage == kP2Stages) {
+        if (++stage == C::kStages) {
           stage = 0;
           phase ^= 1u;
         }
       }
       if (ok) {
-        commit_pair(accf0);
-        commit_pair(accf1);
+        commit_pair(accf[buf][0]);
+        commit_pair(accf[buf][1]);
       }
     }
     if (!ok && issued) {
@@ -311,7 +341,8 @@ __global__ void __launch_bounds__(kP2Threads, 1)
     Segments seg = seg0;
     int u, kb0, kb1;
     while (seg.next(u, kb0, kb1)) {
-      if (!wait_cluster(acc_full, it & 1, abort_flag, a.hdr, kSiteEpiAccFull, a.timeout_ns)) break;
+      const int buf = it % C::kBufs;
+      if (!wait_cluster(&acc_full[buf], (it / C::kBufs) & 1, abort_flag, a.hdr, kSiteEpiAccFull, a.timeout_ns)) break;
       ++it;
       tc_fence_after();
       int4 ch;
@@ -319,7 +350,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       unit_coords<true, kPairTokens>(a, u, ch, mt);
       const int p0 = ch.y, nv = ch.z;
       const int rb = static_cast<int>(rank) * kP2Tok + q * 32;   // first chunk row of this warp's block
-      const uint32_t th = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t th = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
       if constexpr (!kW2) {
         const int i0 = mt * 2 * kP2Rows;
         for (int c0 = hx * kP2Rows; c0 < (rb < nv ? (hx + 1) * kP2Rows : 0); c0 += 16) {
@@ -354,8 +385,9 @@ __global__ void __launch_bounds__(kP2Threads, 1)
         const int f = rb + lane < nv ? a.perm[p0 + rb + lane] : -1;
         const bool valid = f >= 0 && f < a.num_assign;
         const float wt = valid ? a.topk_w[f] : 0.f;
-        const int h0 = mt * 4 * kP2Rows;
-        for (int c0 = hx * 2 * kP2Rows; c0 < (rb < nv ? (hx + 1) * 2 * kP2Rows : 0); c0 += 16) {
+        const int h0 = mt * C::kSlice;
+        constexpr int kHalf = C::kAccCols / 2;   // columns per warp half
+        for (int c0 = hx * kHalf; c0 < (rb < nv ? (hx + 1) * kHalf : 0); c0 += 16) {
           float v[16];
           tmem_ld16_wait(th + c0, v);
 #pragma unroll
@@ -378,7 +410,7 @@ __global__ void __launch_bounds__(kP2Threads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) arrive_cluster(acc_empty0);
+      if (lane == 0) arrive_cluster(acc_empty0[buf]);
     }
   }
 
@@ -404,14 +436,15 @@ bool w2_pair2sm_supported(int H, bool fp8) {
   return v == 1 && !fp8 && H % (4 * kP2Rows) == 0;
 }
 
-template <bool kW2>
+template <bool kW2, bool kDB>
 static cudaError_t launch_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
                                   cudaStream_t st) {
-  auto kern = gemm_pair2sm_kernel<kW2>;
-  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), kP2Smem);
+  using C = P2<kW2, kDB>;
+  auto kern = gemm_pair2sm_kernel<kW2, kDB>;
+  cudaError_t err = set_smem_limit_once(reinterpret_cast<const void*>(kern), C::kSmem);
   if (err != cudaSuccess) return err;
   // as many CTA pairs as can be resident at once (one CTA per SM)
-  static int pairs_cache[64] = {0};
+  static int pairs_cache[64] = {0};   // per device (and per form: one instance per template)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
   int pairs = (dev >= 0 && dev < 64) ? pairs_cache[dev] : 0;
@@ -419,7 +452,7 @@ static cudaError_t launch_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, 
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(2 * (max_ctas / 2));
     q.blockDim = dim3(kP2Threads);
-    q.dynamicSmemBytes = kP2Smem;
+    q.dynamicSmemBytes = C::kSmem;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
     qa[0].val.clusterDim.x = 2;
@@ -437,7 +470,7 @@ static cudaError_t launch_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs);
   cfg.blockDim = dim3(kP2Threads);
-  cfg.dynamicSmemBytes = kP2Smem;
+  cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -449,19 +482,21 @@ static cudaError_t launch_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, 
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   GemmArgs g = a;
-  // slices per CTA pair: 256 rows of I (gate/up) or 512 rows of H (down)
-  g.mtiles = kW2 ? a.w_rows_per_expert / (4 * kP2Rows) : a.up_offset / (2 * kP2Rows);
+  // slices per CTA pair: 256 rows of I (gate/up) or C::kSlice rows of H (down)
+  g.mtiles = kW2 ? a.w_rows_per_expert / C::kSlice : a.up_offset / C::kSlice;
   return cudaLaunchKernelEx(&cfg, kern, tw, tx, g);
 }
 
 cudaError_t launch_w13_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
                                cudaStream_t st) {
-  return launch_pair2sm<false>(tw, tx, a, max_ctas, st);
+  return launch_pair2sm<false, false>(tw, tx, a, max_ctas, st);
 }
 
 cudaError_t launch_w2_pair2sm(const CUtensorMap& tw, const CUtensorMap& tx, const GemmArgs& a, int max_ctas,
                               cudaStream_t st) {
-  return launch_pair2sm<true>(tw, tx, a, max_ctas, st);
+  static const int db = env_on("MOE_W2_2SM_DB");
+  if (db) return launch_pair2sm<true, true>(tw, tx, a, max_ctas, st);
+  return launch_pair2sm<true, false>(tw, tx, a, max_ctas, st);
 }
 
 }  // namespace moe
