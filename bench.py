@@ -297,15 +297,16 @@ SWAP_MAX_TOKENS = 64   # the library's default swap-AB / normal threshold (token
 
 
 def launches_per_step(wl, T):
-    """Kernels one layer call launches: router (logits and top-k; at decode
-    sizes the top-k's last CTA aligns, else one or two align grids), gather,
-    w13 and w2 GEMMs (one per orientation in use, or one fused launch for
-    bf16 decode batches; the FP8 requantisation closes the last w13 launch),
-    and the combine pass."""
+    """Kernels one layer call launches: router (logits and top-k), the align
+    (one grid, or two slice grids from T*k = 8192; with MOE_FUSE_ALIGN=1 the
+    top-k's last CTA aligns decode-sized calls), gather, w13 and w2 GEMMs
+    (one per orientation in use, or one fused launch for bf16 decode
+    batches; the FP8 requantisation closes the last w13 launch), and the
+    combine pass."""
     any_normal = T > SWAP_MAX_TOKENS and wl["H"] % 256 == 0
     A = T * wl["top_k"]
-    # logits, top-k (decode-sized calls: its last CTA aligns), else align (one or two grids)
-    n_route = 2 + (0 if (A < 8192 and wl["E"] <= 256) else (2 if A >= 8192 else 1))
+    fuse_align = os.environ.get("MOE_FUSE_ALIGN", "0") == "1" and A < 8192 and wl["E"] <= 256
+    n_route = 2 + (0 if fuse_align else (2 if A >= 8192 else 1))
     # bf16 decode batches (T <= 32): both GEMMs in one launch; then the combine pass
     fused_ffn = wl["dtype"] == "bf16" and T <= 32 and os.environ.get("MOE_FUSED_FFN", "1") != "0"
     n_gemm = 1 if fused_ffn else 2 * (2 if any_normal else 1)

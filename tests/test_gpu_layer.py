@@ -418,3 +418,18 @@ def test_route_tests_on_tensor_core_tier(cuda_ok):
                         "route and not tensor_core_tier", "-p", "no:cacheprovider"],
                        env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+def test_align_folded_into_top_k(cuda_ok):
+    """The decode-sized layer again with the align run by the top-k kernel's
+    last CTA (MOE_FUSE_ALIGN=1, fixed per process, so in a child process):
+    routing bit-exact and outputs within the bound, as with the separate
+    align launch."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_FUSE_ALIGN="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", __file__, "-m", "gpu", "-x", "-q", "-k",
+                        "forward_parity_bf16", "-p", "no:cacheprovider"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
