@@ -39,6 +39,15 @@
 //             CTA's barrier);
 //   acc_full  each CTA's own: rank 0 commits after the unit's last K atom;
 //   acc_empty rank 0's: one arrival per epilogue warp of both CTAs.
+// The producers' arrivals stay inside the CTA: rank 0 alone arms full[s]
+// with the bytes of both CTAs' copies (a cluster-scope release on every
+// stage, as in a two-arrival form, cost about a microsecond per stage and
+// left the ring serialised).
+// Every wait is bounded (wait_cluster, mbar_wait): a CTA that gives up
+// raises its abort flag and leaves its loops (rank 0's MMA issuer first
+// waits, again bounded, for the MMAs it has in flight; copies in flight land
+// within microseconds, long before a wait gives up), and both CTAs meet at
+// the final cluster barrier before TMEM is released.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
