@@ -62,8 +62,9 @@ struct RouterArgs {
   float* partials;        // GEMM partial tiles for the tensor-core logits (NULL: whole units)
 };
 struct AlignArgs;
-// fuse_align non-NULL: a decode-sized call may run logits, top-k and align in
-// one launch (then *fused is set and the align must not be launched again).
+// fuse_align non-NULL and MOE_FUSE_ALIGN=1: a decode-sized call lets the
+// top-k kernel's last CTA run the align (then *fused is set and the align
+// must not be launched again); by default the align is its own launch.
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t st, const AlignArgs* fuse_align = nullptr,
                           bool* fused = nullptr);
 // The top-k of logits from the tensor cores (logits, norms and amax already
