@@ -83,6 +83,10 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
   const int cend = mode == 0 ? A : min(A, cbeg + slice);
   const bool lead = mode == 0 || (mode == 2 && blockIdx.x == 0);   // writes the shared outputs
 
+  // FP8 activation scale inputs, requested now so they arrive during the histogram
+  float m_pre = 0.f;
+  if (lead && a.amax_tok != nullptr)
+    for (int t = threadIdx.x; t < a.T; t += blockDim.x) m_pre = fmaxf(m_pre, __ldcg(a.amax_tok + t));
   for (int i = threadIdx.x; i < NW * E; i += blockDim.x) hist[i] = 0;
   if (a.gemm_flags != nullptr && (mode == 0 || (mode == 1 && blockIdx.x == 0)))
     for (int i = threadIdx.x; i < a.n_gemm_flags; i += blockDim.x) a.gemm_flags[i] = 0;
@@ -94,12 +98,17 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
   const int kbits = 32 - __clz(E);   // bits of the keys 0..E (E = "no expert")
   const int per = (cend - cbeg + NW - 1) / NW;
   const int beg = min(cend, cbeg + warp * per), end = min(cend, beg + per);
+  // a slice of at most one batch per warp (decode-sized calls) keeps its ids
+  // in registers for the scatter pass instead of loading them again
+  const bool one_batch = per <= 32 * kBatch;
+  int keep[kBatch];
   for (int base = beg; base < end; base += 32 * kBatch) {
     int ev[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int f = base + 32 * u + lane;
       ev[u] = f < end ? __ldcg(a.topk_ids + f) : -1;
+      keep[u] = ev[u];
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -160,7 +169,7 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int f = base + 32 * u + lane;
-      ev[u] = f < end ? __ldcg(a.topk_ids + f) : -1;
+      ev[u] = one_batch ? keep[u] : (f < end ? __ldcg(a.topk_ids + f) : -1);
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
@@ -219,8 +228,7 @@ __device__ __forceinline__ void align_cta(const AlignArgs& a, int mode, int slic
 
   // FP8 activation scale: s1 = amax / 448 (one IEEE fp32 division); amax == 0 -> 1
   if (a.amax_tok != nullptr) {
-    float m = 0.f;
-    for (int t = threadIdx.x; t < a.T; t += blockDim.x) m = fmaxf(m, __ldcg(a.amax_tok + t));
+    float m = m_pre;
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, d));
     if (lane == 0) famax[warp] = m;
